@@ -1,0 +1,153 @@
+/*
+ * rq.h -- C ABI of librq: blockwise rotated scalar quantization and the QJL
+ * 1-bit sketch on NVIDIA B200 (sm_100a).
+ *
+ * Operations (sources: the eliza quantization README, sections "PolarQuant",
+ * "TurboQuant" and "QJL", each "Algorithm in one paragraph"; the qjl_apply.py
+ * source text, `_build_jl_projections` and `_qjl_decode_keys`; the turbopress
+ * 0.4.2 project description, "Package layout" and "Findings"):
+ *
+ *   quantize    x (blocks of d contiguous values) -> per-block fp16 L2 norm and
+ *               per-coordinate index of the nearest centroid of
+ *               y = H D x / ||x||, H the d x d Sylvester Hadamard matrix (unnormalised,
+ *               so y is the orthonormal rotation of x/||x|| scaled by sqrt(d)), D an
+ *               optional seeded +-1 diagonal.
+ *   dequantize  codes, norms -> x^ = n16 * D * H c / d, c_j = centroid[code_j]
+ *               (centroid lookup, divide by sqrt(d), inverse rotation, rescale).
+ *   QJL sketch  v -> sign(S v) packed 8 per byte and fp16 ||v||, S an m x d
+ *               seeded Gaussian matrix.
+ *   QJL score   <q, k> ~ (n16/d) <H D q, c> + sqrt(pi/2)/m * ||r|| * <S q, sign(S r)>
+ *               (first term only when the key carries a first-stage code).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named x, codes, norms, out, proj, signs, scores, q and workspace
+ *     are DEVICE pointers owned by the caller; `centroids` is a HOST pointer.
+ *     The library keeps no pointer after a call returns, allocates no device
+ *     memory and keeps no global state.
+ *   - Every call validates its arguments on the host, then enqueues its
+ *     kernels asynchronously on `stream` (0 = legacy default stream) and
+ *     returns.  Kernel faults surface at the caller's next synchronisation.
+ *   - Return value: RQ_OK or a negative rq_status; on error nothing is enqueued.
+ *   - Device pointers must be 16-byte aligned.
+ *   - d (block size / head dim) is a power of two in {64, 128, 256, 512}
+ *     ("--block-size N, must be a power of 2" and "head_dim must be a power of
+ *     2" on the pages); n must be a multiple of d.
+ *   - Arithmetic is fp32 in one canonical order so results are reproducible
+ *     bit for bit: the norm is the pairwise (recursive halving) fp32 sum of
+ *     fp32 squares with a correctly rounded sqrt; the Hadamard transform runs
+ *     radix-2 stages h = 1, 2, ..., d/2; y_j = v_j * (1/n32) (y = 0 when n32 = 0);
+ *     code = #{k : t_k < y} with t_k = fl32(0.5 * fl32(c_k + c_k+1)) (ties go to
+ *     the lower index); x^_j = s_j * (w_j * (n16 / d)), output rounded to
+ *     nearest even.  Norms round to fp16 and saturate at 65504.
+ *   - Code storage, one field of rq_code_bytes(d, bits, layout) bytes per block:
+ *     RQ_CODES_INT8: one byte per coordinate; RQ_CODES_PACKED: code j of the
+ *     block occupies bits [j*bits, (j+1)*bits) of the field, least significant
+ *     bit first (two codes per byte at 4 bits, four at 2 bits).
+ *   - Sign diagonal: s_j = -1 iff bit (j mod 64) of output floor(j/64) of the
+ *     SplitMix64 stream with initial state sign_seed is set; one diagonal per
+ *     call, shared by every block.
+ *   - Sign sketch storage: m/8 bytes per vector; coordinate i is bit (i mod 8)
+ *     of byte i/8; bit 1 <-> P_i >= 0 (sign +1).
+ */
+#ifndef RQ_H
+#define RQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *rq_stream_t;   /* the same handle as cudaStream_t */
+
+typedef enum {
+    RQ_OK = 0,
+    RQ_EINVAL = -1,        /* bad size, NULL pointer, unsorted/non-finite table, ... */
+    RQ_EALIGN = -2,        /* a device pointer is not 16-byte aligned */
+    RQ_ESIZE = -3,         /* a size does not fit the kernels' index arithmetic */
+    RQ_EUNSUPPORTED = -4,  /* valid but not implemented (d, bits, m, dtype combination) */
+    RQ_ECUDA = -5          /* a CUDA runtime call failed (launch error, ...) */
+} rq_status;
+
+typedef enum { RQ_F16 = 0, RQ_BF16 = 1 } rq_dtype;
+typedef enum { RQ_CODES_PACKED = 0, RQ_CODES_INT8 = 1 } rq_layout;
+
+/* Human-readable name of a status code (static string). */
+const char *rq_status_string(int status);
+
+/* Bytes of code storage for n values in blocks of d: (n/d) * (d*bits/8) packed,
+ * n for int8.  Returns -1 on invalid arguments. */
+int64_t rq_code_bytes(int64_t n, int d, int bits, rq_layout layout);
+
+/* Lloyd-Max reconstruction levels for N(0,1) at `bits` (1..8), ascending,
+ * written to the HOST array centroids_out[2^bits] as fp32.  Computed by the
+ * conditional-expectation fixed point in fp64 (PolarQuant paragraph: "Lloyd-Max
+ * optimal centroids for N(0,1) ... iterative conditional-expectation
+ * algorithm"), made exactly odd-symmetric, then rounded to fp32. */
+rq_status rq_lloyd_max(int bits, float *centroids_out);
+
+/* Quantize n values of x (dtype fp16/bf16, n % d == 0, blocks contiguous).
+ *   bits 1..8 (int8 layout) or 1..8 (packed); centroids: HOST, 2^bits finite
+ *   strictly ascending fp32 values.
+ *   codes: rq_code_bytes(n, d, bits, layout) bytes; norms: n/d fp16.
+ *   use_signs = 0 means D = I (sign_seed ignored). */
+rq_status rq_quantize(const void *x, rq_dtype dtype, int64_t n, int d, int bits, rq_layout layout,
+                      int use_signs, uint64_t sign_seed, const float *centroids,
+                      void *codes, uint16_t *norms, rq_stream_t stream);
+
+/* Reconstruct n values into out (out_dtype) from codes and fp16 norms written
+ * by rq_quantize with the same d, bits, layout, signs and centroids. */
+rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int d, int bits,
+                        rq_layout layout, int use_signs, uint64_t sign_seed, const float *centroids,
+                        void *out, rq_dtype out_dtype, rq_stream_t stream);
+
+/* Quantize (as rq_quantize) and sketch the first-stage residual in the same
+ * pass (PolarQuant paragraph: "optionally append a 1-bit QJL residual"; the
+ * two-stage TurboQuant-style key code):
+ *   r = x - x^32 (fp32, x^32 the reconstruction before output rounding),
+ *   qjl_norms[b] = fp16(||r||) (canonical fp32 norm),
+ *   qjl_signs[b][m/8] = sign bits of S r_bf16, r_bf16 = bf16(r), S = proj.
+ *   proj: m x d bf16 row-major (qjl_make_projection); m % 8 == 0, 8 <= m <= 512. */
+rq_status rq_quantize_qjl(const void *x, rq_dtype dtype, int64_t n, int d, int bits, rq_layout layout,
+                          int use_signs, uint64_t sign_seed, const float *centroids,
+                          int m, const void *proj, void *codes, uint16_t *norms,
+                          uint8_t *qjl_signs, uint16_t *qjl_norms, rq_stream_t stream);
+
+/* Write the m x d JL matrix S[i][j] = round16(fp32(gauss(seed, i*d + j))) to
+ * proj (dtype bf16 or fp16, row-major).  gauss(seed, k) is the Box-Muller
+ * normal sqrt(-2 ln u1) cos(2 pi u2) with u1 = (w_2k >> 11 + 1) 2^-53,
+ * u2 = (w_2k+1 >> 11) 2^-53, w_i output i of SplitMix64 seeded with `seed`
+ * (qjl_apply.py `_build_jl_projections`: plain N(0,1) entries, no QR). */
+rq_status qjl_make_projection(uint64_t seed, int m, int d, rq_dtype dtype, void *proj, rq_stream_t stream);
+
+/* QJL sketch of n_vec vectors x[n_vec][d] (dtype = proj dtype):
+ * signs[n_vec][m/8] of S x, norms[n_vec] = fp16(||x||) (QJL paragraph:
+ * "extract ||k||", "take the sign of each sketch coordinate, packing 8 signs
+ * into one uint8"). */
+rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m, const void *proj,
+                     uint8_t *signs, uint16_t *norms, rq_stream_t stream);
+
+/* Device workspace qjl_score needs for G groups of n_q queries (bytes). */
+size_t qjl_score_workspace_bytes(int64_t G, int n_q, int d, int m);
+
+/* Inner-product scores of n_q queries against T compressed keys per group
+ * (group = batch x kv-head; the n_q queries of a group share its keys, the
+ * grouped-query shape):
+ *   q: bf16 [G][n_q][d]; proj: m x d (proj_dtype); signs [G][T][m/8];
+ *   sk_norms fp16 [G][T] (the norm the sketch was taken of);
+ *   codes/norms: first-stage codes [G][T] blocks of d and fp16 norms, or
+ *   codes == NULL for the pure QJL score;
+ *   scores: fp32 [G][n_q][T];
+ *   workspace: qjl_score_workspace_bytes(G, n_q, d, m) bytes of device memory
+ *   (overwritten). */
+rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void *proj, rq_dtype proj_dtype,
+                    const uint8_t *signs, const uint16_t *sk_norms, int64_t T,
+                    const void *codes, const uint16_t *norms, int bits, rq_layout layout,
+                    int use_signs, uint64_t sign_seed, const float *centroids,
+                    float *scores, void *workspace, size_t workspace_bytes, rq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RQ_H */

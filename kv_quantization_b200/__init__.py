@@ -1,0 +1,11 @@
+"""kv_quantization_b200 -- B200-native rotated scalar quantization and QJL sketching.
+
+The product is the C-ABI library ``librq.so`` (include/rq.h) built from
+``csrc/`` for sm_100a; ``_lib`` is its ctypes binding (same function names),
+``synth`` the seeded input recipes, ``build`` the nvcc build step.
+"""
+from ._lib import (  # noqa: F401
+    RQ_BF16, RQ_CODES_INT8, RQ_CODES_PACKED, RQ_F16, RQError, lib, qjl_make_projection, qjl_score,
+    qjl_score_workspace_bytes, qjl_sketch, rq_code_bytes, rq_dequantize, rq_lloyd_max, rq_quantize,
+    rq_quantize_qjl, status_string,
+)

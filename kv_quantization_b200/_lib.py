@@ -1,0 +1,159 @@
+"""ctypes binding of librq (include/rq.h), argument marshalling only.
+
+Every function here has the name of the C entry point it calls and forwards
+its arguments unchanged: device buffers are torch CUDA tensors (passed by
+data pointer), ``centroids`` is a host float32 array, ``stream`` defaults to
+torch's current CUDA stream.  All arithmetic runs in librq's kernels; a
+missing or unloadable librq.so raises immediately -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librq.so")
+
+RQ_F16, RQ_BF16 = 0, 1
+RQ_CODES_PACKED, RQ_CODES_INT8 = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+class RQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+def lib() -> C.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"librq.so not built ({LIB_PATH}); run python -m kv_quantization_b200.build")
+            L = C.CDLL(LIB_PATH)
+            vp, i64, i32, u64, sz = C.c_void_p, C.c_int64, C.c_int, C.c_uint64, C.c_size_t
+            fp = C.POINTER(C.c_float)
+            sig = {
+                "rq_status_string": (C.c_char_p, [i32]),
+                "rq_code_bytes": (i64, [i64, i32, i32, i32]),
+                "rq_lloyd_max": (i32, [i32, fp]),
+                "rq_quantize": (i32, [vp, i32, i64, i32, i32, i32, i32, u64, fp, vp, vp, vp]),
+                "rq_dequantize": (i32, [vp, vp, i64, i32, i32, i32, i32, u64, fp, vp, i32, vp]),
+                "rq_quantize_qjl": (i32, [vp, i32, i64, i32, i32, i32, i32, u64, fp, i32, vp, vp, vp, vp, vp, vp]),
+                "qjl_make_projection": (i32, [u64, i32, i32, i32, vp, vp]),
+                "qjl_sketch": (i32, [vp, i32, i64, i32, i32, vp, vp, vp, vp]),
+                "qjl_score_workspace_bytes": (sz, [i64, i32, i32, i32]),
+                "qjl_score": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32, u64,
+                                    fp, vp, vp, sz, vp]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def exported_symbols():
+    """Names this binding expects librq.so to export."""
+    return ["rq_status_string", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
+            "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score"]
+
+
+def status_string(status: int) -> str:
+    return lib().rq_status_string(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != 0:
+        raise RQError(fn, status)
+
+
+def _dev(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _table(centroids):
+    c = np.ascontiguousarray(np.asarray(centroids, dtype=np.float32))
+    return c, c.ctypes.data_as(C.POINTER(C.c_float))
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return RQ_BF16
+    if t.dtype == torch.float16:
+        return RQ_F16
+    raise TypeError(f"expected a bfloat16 or float16 tensor, got {t.dtype}")
+
+
+# ------------------------------------------------------------------ entry points
+
+def rq_code_bytes(n: int, d: int, bits: int, layout: int) -> int:
+    return lib().rq_code_bytes(n, d, bits, layout)
+
+
+def rq_lloyd_max(bits: int) -> np.ndarray:
+    out = np.zeros(1 << bits, np.float32)
+    _check("rq_lloyd_max", lib().rq_lloyd_max(bits, out.ctypes.data_as(C.POINTER(C.c_float))))
+    return out
+
+
+def rq_quantize(x, d, bits, layout, use_signs, sign_seed, centroids, codes, norms, stream=None, n=None):
+    c, cp = _table(centroids)
+    _check("rq_quantize", lib().rq_quantize(_dev(x), _dtype_code(x), x.numel() if n is None else n, d, bits, layout,
+                                            int(use_signs), sign_seed, cp, _dev(codes), _dev(norms), _stream(stream)))
+
+
+def rq_dequantize(codes, norms, n, d, bits, layout, use_signs, sign_seed, centroids, out, stream=None):
+    c, cp = _table(centroids)
+    _check("rq_dequantize", lib().rq_dequantize(_dev(codes), _dev(norms), n, d, bits, layout, int(use_signs),
+                                                sign_seed, cp, _dev(out), _dtype_code(out), _stream(stream)))
+
+
+def rq_quantize_qjl(x, d, bits, layout, use_signs, sign_seed, centroids, m, proj, codes, norms, qjl_signs,
+                    qjl_norms, stream=None, n=None):
+    c, cp = _table(centroids)
+    _check("rq_quantize_qjl", lib().rq_quantize_qjl(
+        _dev(x), _dtype_code(x), x.numel() if n is None else n, d, bits, layout, int(use_signs), sign_seed, cp,
+        m, _dev(proj), _dev(codes), _dev(norms), _dev(qjl_signs), _dev(qjl_norms), _stream(stream)))
+
+
+def qjl_make_projection(seed, m, d, proj, stream=None):
+    _check("qjl_make_projection", lib().qjl_make_projection(seed, m, d, _dtype_code(proj), _dev(proj),
+                                                            _stream(stream)))
+
+
+def qjl_sketch(x, d, m, proj, signs, norms, stream=None, n_vec=None):
+    nv = x.numel() // d if n_vec is None else n_vec
+    _check("qjl_sketch", lib().qjl_sketch(_dev(x), _dtype_code(x), nv, d, m, _dev(proj), _dev(signs), _dev(norms),
+                                          _stream(stream)))
+
+
+def qjl_score_workspace_bytes(G, n_q, d, m) -> int:
+    return lib().qjl_score_workspace_bytes(G, n_q, d, m)
+
+
+def qjl_score(q, G, n_q, d, m, proj, signs, sk_norms, T, scores, workspace, codes=None, norms=None, bits=0,
+              layout=RQ_CODES_PACKED, use_signs=0, sign_seed=0, centroids=None, stream=None):
+    if centroids is None:
+        cp = None
+    else:
+        c, cp = _table(centroids)
+    _check("qjl_score", lib().qjl_score(
+        _dev(q), G, n_q, d, m, _dev(proj), _dtype_code(proj), _dev(signs), _dev(sk_norms), T, _dev(codes),
+        _dev(norms), bits, layout, int(use_signs), sign_seed, cp, _dev(scores), _dev(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))

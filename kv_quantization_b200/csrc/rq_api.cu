@@ -1,0 +1,362 @@
+// rq_api.cu -- the C ABI of librq (declared in include/rq.h): argument
+// validation, per-call tables (Lloyd-Max levels, decision thresholds, the
+// exact search LUT, the sign diagonal) and kernel launches.  No device memory
+// is allocated here; every table travels to the kernels as a by-value
+// parameter block.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "rq.h"
+#include "rq_kernels.h"
+
+using rq::QuantTables;
+
+namespace {
+
+bool pow2_d(int d) { return d == 64 || d == 128 || d == 256 || d == 512; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+uint64_t splitmix64(uint64_t seed, uint64_t k)
+{
+    uint64_t z = seed + (k + 1ull) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// Total order on finite floats as integers (for searching the float line).
+int64_t fkey(float f)
+{
+    int32_t i;
+    std::memcpy(&i, &f, 4);
+    return i >= 0 ? (int64_t)i : (int64_t)INT32_MIN - (int64_t)i;
+}
+float keyf(int64_t k)
+{
+    int32_t i = k >= 0 ? (int32_t)k : (int32_t)((int64_t)INT32_MIN - k);
+    float f;
+    std::memcpy(&f, &i, 4);
+    return f;
+}
+
+// The device's cell function, evaluated with the same IEEE fma.
+int lut_cell(float y, float a, float b, int cells)
+{
+    const float f = std::fmaf(y, a, b);
+    uint32_t fb, mb;
+    const float magic = rq::kLutMagic;
+    std::memcpy(&fb, &f, 4);
+    std::memcpy(&mb, &magic, 4);
+    int c = (int)(fb - mb);
+    return c < 0 ? 0 : (c > cells - 1 ? cells - 1 : c);
+}
+
+// Build the exact LUT: each cell's set of y values is an interval; a cell may
+// hold at most one decision threshold.  Returns false when no grid of at most
+// kMaxLutCells cells separates the thresholds (the kernels then binary-search).
+bool build_lut(const float *t, int nb, QuantTables &T)
+{
+    if (nb < 1) return false;
+    double min_gap = INFINITY;
+    for (int k = 0; k + 1 < nb; ++k) min_gap = std::fmin(min_gap, (double)t[k + 1] - (double)t[k]);
+    if (!(min_gap > 0)) return false;
+    if (!std::isfinite(min_gap)) min_gap = 1.0;
+    const double span = (double)t[nb - 1] - (double)t[0];
+    const float lo_lim = -1.0e5f, hi_lim = 1.0e5f;   // |y| <= sqrt(d) for finite input
+    for (int attempt = 0; attempt < 64; ++attempt) {
+        const float a = (float)((1.0 + 0.125 * attempt) / min_gap);
+        const int cells = (int)std::ceil(span * (double)a) + 4;
+        if (cells > rq::kMaxLutCells || !(a > 0) || !std::isfinite(a)) return false;
+        const float b0 = (float)(2.0 - std::floor((double)t[0] * (double)a));
+        const float b = rq::kLutMagic + b0;
+        if (std::fabs((double)b0) + std::fabs((double)a) * 1.0e5 > 4.0e6) return false;
+        // ylo[j]: smallest float y in [lo_lim, hi_lim] with cell(y) >= j.
+        std::vector<float> ylo(cells + 1);
+        ylo[0] = -INFINITY;
+        ylo[cells] = INFINITY;
+        for (int j = 1; j < cells; ++j) {
+            int64_t lo = fkey(lo_lim), hi = fkey(hi_lim);
+            if (lut_cell(keyf(hi), a, b, cells) < j) { ylo[j] = INFINITY; continue; }
+            while (lo < hi) {
+                const int64_t mid = lo + (hi - lo) / 2;
+                if (lut_cell(keyf(mid), a, b, cells) >= j) hi = mid; else lo = mid + 1;
+            }
+            ylo[j] = keyf(lo);
+        }
+        bool ok = true;
+        for (int j = 0; j < cells && ok; ++j) {
+            int below = 0, inside = 0;
+            float cand = INFINITY;
+            for (int k = 0; k < nb; ++k) {
+                if (t[k] < ylo[j]) ++below;
+                else if (t[k] < ylo[j + 1]) { ++inside; cand = t[k]; }
+            }
+            if (inside > 1) ok = false;
+            T.lut_k[j] = (uint32_t)below;
+            T.lut_t[j] = inside ? cand : INFINITY;
+        }
+        if (ok) {
+            T.lut_a = a;
+            T.lut_b = b;
+            T.lut_cells = cells;
+            return true;
+        }
+    }
+    return false;
+}
+
+// Validate a host centroid table and fill the per-call tables.
+rq_status make_tables(const float *centroids, int bits, int d, int use_signs, uint64_t sign_seed,
+                      QuantTables &T)
+{
+    std::memset(&T, 0, sizeof(T));
+    const int K = 1 << bits;
+    if (!centroids) return RQ_EINVAL;
+    for (int k = 0; k < K; ++k) {
+        if (!std::isfinite(centroids[k]) || std::fabs(centroids[k]) > 1.0e4f) return RQ_EINVAL;
+        if (k > 0 && !(centroids[k] > centroids[k - 1])) return RQ_EINVAL;
+        T.centroid[k] = centroids[k];
+    }
+    T.levels = K;
+    for (int k = 0; k + 1 < K; ++k) {
+        const float s = centroids[k] + centroids[k + 1];
+        T.bound[k] = 0.5f * s;
+    }
+    T.bound[K - 1] = INFINITY;
+    if (!build_lut(T.bound, K - 1, T)) T.lut_cells = 0;
+    if (use_signs) {
+        for (int w = 0; w < d / 64; ++w) {
+            const uint64_t r = splitmix64(sign_seed, (uint64_t)w);
+            T.sign_words[2 * w] = (uint32_t)(r & 0xffffffffu);
+            T.sign_words[2 * w + 1] = (uint32_t)(r >> 32);
+        }
+    }
+    return RQ_OK;
+}
+
+rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ECUDA; }
+
+// Lloyd-Max iteration for N(0,1): levels are conditional means of their cells,
+// thresholds are midpoints.  phi / Phi differences on the tail side.
+double npdf(double t) { return std::isinf(t) ? 0.0 : std::exp(-0.5 * t * t) * 0.39894228040143267794; }
+double cell_mass(double a, double b)
+{
+    const double r = 0.70710678118654752440;
+    if (a >= 0.0) return 0.5 * (std::erfc(a * r) - std::erfc(b * r));
+    if (b <= 0.0) return 0.5 * (std::erfc(-b * r) - std::erfc(-a * r));
+    return 1.0 - 0.5 * std::erfc(-a * r) - 0.5 * std::erfc(b * r);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *rq_status_string(int status)
+{
+    switch (status) {
+    case RQ_OK: return "RQ_OK";
+    case RQ_EINVAL: return "RQ_EINVAL: invalid argument";
+    case RQ_EALIGN: return "RQ_EALIGN: device pointer not 16-byte aligned";
+    case RQ_ESIZE: return "RQ_ESIZE: size out of range";
+    case RQ_EUNSUPPORTED: return "RQ_EUNSUPPORTED: unsupported combination";
+    case RQ_ECUDA: return "RQ_ECUDA: CUDA runtime error";
+    default: return "unknown rq_status";
+    }
+}
+
+int64_t rq_code_bytes(int64_t n, int d, int bits, rq_layout layout)
+{
+    if (!pow2_d(d) || bits < 1 || bits > 8 || n < 0 || n % d) return -1;
+    if (layout == RQ_CODES_INT8) return n;
+    if (layout != RQ_CODES_PACKED) return -1;
+    return (n / d) * ((int64_t)d * bits / 8);
+}
+
+rq_status rq_lloyd_max(int bits, float *centroids_out)
+{
+    if (bits < 1 || bits > 8 || !centroids_out) return RQ_EINVAL;
+    const int K = 1 << bits;
+    std::vector<double> c(K), t(K + 1);
+    for (int i = 0; i < K; ++i) c[i] = 4.0 * (2.0 * i + 1.0 - K) / K;   // sorted start in [-4, 4]
+    for (int it = 0; it < 1000000; ++it) {
+        t[0] = -INFINITY;
+        t[K] = INFINITY;
+        for (int i = 1; i < K; ++i) t[i] = 0.5 * (c[i - 1] + c[i]);
+        double worst = 0.0;
+        for (int i = 0; i < K; ++i) {
+            const double nc = (npdf(t[i]) - npdf(t[i + 1])) / cell_mass(t[i], t[i + 1]);
+            worst = std::fmax(worst, std::fabs(nc - c[i]));
+            c[i] = nc;
+        }
+        if (worst < 1e-13) break;
+    }
+    for (int i = 0; i < K / 2; ++i) {
+        const double a = 0.5 * (c[K - 1 - i] - c[i]);
+        c[i] = -a;
+        c[K - 1 - i] = a;
+    }
+    for (int i = 0; i < K; ++i) centroids_out[i] = (float)c[i];
+    return RQ_OK;
+}
+
+static rq_status check_common(int64_t n, int d, int bits, rq_layout layout)
+{
+    if (!pow2_d(d)) return (d > 0 && (d & (d - 1)) == 0) ? RQ_EUNSUPPORTED : RQ_EINVAL;
+    if (bits < 1 || bits > 8) return RQ_EINVAL;
+    if (layout != RQ_CODES_PACKED && layout != RQ_CODES_INT8) return RQ_EINVAL;
+    if (n < 0 || n % d) return RQ_EINVAL;
+    if (n > ((int64_t)1 << 40)) return RQ_ESIZE;
+    return RQ_OK;
+}
+
+static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, int bits, rq_layout layout,
+                               int use_signs, uint64_t sign_seed, const float *centroids, int m,
+                               const void *proj, void *codes, uint16_t *norms, uint8_t *qjl_signs,
+                               uint16_t *qjl_norms, cudaStream_t stream)
+{
+    rq_status s = check_common(n, d, bits, layout);
+    if (s) return s;
+    if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
+    const bool qjl = qjl_signs != nullptr || qjl_norms != nullptr || proj != nullptr;
+    if (qjl && (!qjl_signs || !qjl_norms || !proj || m < 8 || m > 512 || m % 8)) return RQ_EINVAL;
+    if (n == 0) return RQ_OK;
+    if (!x || !codes || !norms) return RQ_EINVAL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(norms)) return RQ_EALIGN;
+    if (qjl && (!aligned16(proj) || !aligned16(qjl_signs) || !aligned16(qjl_norms))) return RQ_EALIGN;
+    QuantTables T;
+    s = make_tables(centroids, bits, d, use_signs, sign_seed, T);
+    if (s) return s;
+    rq::QuantArgs a{};
+    a.x = x; a.nblocks = n / d; a.d = d; a.pw = layout == RQ_CODES_INT8 ? 8 : bits; a.bf16 = dtype == RQ_BF16;
+    a.tables = &T; a.codes = codes; a.norms = norms;
+    a.m = qjl ? m : 0; a.proj = proj; a.qsigns = qjl_signs; a.qnorms = qjl_norms;
+    a.num_sms = num_sms();
+    if (a.num_sms <= 0) return RQ_ECUDA;
+    return cuda_status(rq::launch_quantize(a, stream));
+}
+
+rq_status rq_quantize(const void *x, rq_dtype dtype, int64_t n, int d, int bits, rq_layout layout,
+                      int use_signs, uint64_t sign_seed, const float *centroids,
+                      void *codes, uint16_t *norms, rq_stream_t stream)
+{
+    return quantize_impl(x, dtype, n, d, bits, layout, use_signs, sign_seed, centroids, 0, nullptr, codes, norms,
+                         nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rq_status rq_quantize_qjl(const void *x, rq_dtype dtype, int64_t n, int d, int bits, rq_layout layout,
+                          int use_signs, uint64_t sign_seed, const float *centroids,
+                          int m, const void *proj, void *codes, uint16_t *norms,
+                          uint8_t *qjl_signs, uint16_t *qjl_norms, rq_stream_t stream)
+{
+    if (!proj || !qjl_signs || !qjl_norms) return RQ_EINVAL;
+    return quantize_impl(x, dtype, n, d, bits, layout, use_signs, sign_seed, centroids, m, proj, codes, norms,
+                         qjl_signs, qjl_norms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int d, int bits,
+                        rq_layout layout, int use_signs, uint64_t sign_seed, const float *centroids,
+                        void *out, rq_dtype out_dtype, rq_stream_t stream)
+{
+    rq_status s = check_common(n, d, bits, layout);
+    if (s) return s;
+    if (out_dtype != RQ_F16 && out_dtype != RQ_BF16) return RQ_EINVAL;
+    if (n == 0) return RQ_OK;
+    if (!codes || !norms || !out) return RQ_EINVAL;
+    if (!aligned16(codes) || !aligned16(norms) || !aligned16(out)) return RQ_EALIGN;
+    QuantTables T;
+    s = make_tables(centroids, bits, d, use_signs, sign_seed, T);
+    if (s) return s;
+    rq::DequantArgs a{};
+    a.codes = codes; a.norms = norms; a.nblocks = n / d; a.d = d; a.pw = layout == RQ_CODES_INT8 ? 8 : bits;
+    a.bf16 = out_dtype == RQ_BF16; a.tables = &T; a.out = out;
+    a.num_sms = num_sms();
+    if (a.num_sms <= 0) return RQ_ECUDA;
+    return cuda_status(rq::launch_dequantize(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rq_status qjl_make_projection(uint64_t seed, int m, int d, rq_dtype dtype, void *proj, rq_stream_t stream)
+{
+    if (m < 8 || m > 512 || m % 8 || !pow2_d(d)) return RQ_EINVAL;
+    if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
+    if (!proj) return RQ_EINVAL;
+    if (!aligned16(proj)) return RQ_EALIGN;
+    return cuda_status(rq::launch_projection(seed, m, d, dtype == RQ_BF16, proj,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m, const void *proj,
+                     uint8_t *signs, uint16_t *norms, rq_stream_t stream)
+{
+    if (!pow2_d(d)) return RQ_EINVAL;
+    if (m < 8 || m > 512 || m % 8) return RQ_EINVAL;
+    if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
+    if (n_vec < 0) return RQ_EINVAL;
+    if (n_vec > ((int64_t)1 << 34)) return RQ_ESIZE;
+    if (n_vec == 0) return RQ_OK;
+    if (!x || !proj || !signs || !norms) return RQ_EINVAL;
+    if (!aligned16(x) || !aligned16(proj) || !aligned16(signs) || !aligned16(norms)) return RQ_EALIGN;
+    rq::SketchArgs a{};
+    a.x = x; a.nvec = n_vec; a.d = d; a.m = m; a.bf16 = dtype == RQ_BF16; a.proj = proj; a.signs = signs;
+    a.norms = norms; a.num_sms = num_sms();
+    if (a.num_sms <= 0) return RQ_ECUDA;
+    return cuda_status(rq::launch_sketch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t qjl_score_workspace_bytes(int64_t G, int n_q, int d, int m)
+{
+    if (G < 0 || n_q < 0 || d < 0 || m < 0) return 0;
+    return rq::score_workspace_bytes(G, n_q, d, m);
+}
+
+rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void *proj, rq_dtype proj_dtype,
+                    const uint8_t *signs, const uint16_t *sk_norms, int64_t T_len,
+                    const void *codes, const uint16_t *norms, int bits, rq_layout layout,
+                    int use_signs, uint64_t sign_seed, const float *centroids,
+                    float *scores, void *workspace, size_t workspace_bytes, rq_stream_t stream)
+{
+    if (!pow2_d(d)) return RQ_EINVAL;
+    if (m < 8 || m > 512 || m % 8) return RQ_EINVAL;
+    if (proj_dtype != RQ_F16 && proj_dtype != RQ_BF16) return RQ_EINVAL;
+    if (G < 0 || n_q < 0 || T_len < 0) return RQ_EINVAL;
+    if (G > 65535 || n_q > 32 * 65535 || T_len > ((int64_t)1 << 31)) return RQ_ESIZE;
+    if (G == 0 || n_q == 0 || T_len == 0) return RQ_OK;
+    if (!q || !proj || !signs || !sk_norms || !scores || !workspace) return RQ_EINVAL;
+    if (workspace_bytes < rq::score_workspace_bytes(G, n_q, d, m)) return RQ_ESIZE;
+    if (!aligned16(q) || !aligned16(proj) || !aligned16(signs) || !aligned16(sk_norms) || !aligned16(scores) ||
+        !aligned16(workspace))
+        return RQ_EALIGN;
+    QuantTables T;
+    std::memset(&T, 0, sizeof(T));
+    int pw = 0;
+    if (codes) {
+        rq_status s = check_common(0, d, bits, layout);
+        if (s) return s;
+        if (!norms) return RQ_EINVAL;
+        if (!aligned16(codes) || !aligned16(norms)) return RQ_EALIGN;
+        s = make_tables(centroids, bits, d, use_signs, sign_seed, T);
+        if (s) return s;
+        pw = layout == RQ_CODES_INT8 ? 8 : bits;
+    }
+    rq::ScoreArgs a{};
+    a.q = static_cast<const uint16_t *>(q); a.G = G; a.nq = n_q; a.d = d; a.m = m; a.proj = proj;
+    a.proj_bf16 = proj_dtype == RQ_BF16; a.signs = signs; a.sk_norms = sk_norms; a.T = T_len;
+    a.codes = static_cast<const uint8_t *>(codes); a.norms = norms; a.pw = pw; a.tables = &T;
+    a.scores = scores; a.workspace = static_cast<float *>(workspace); a.num_sms = num_sms();
+    if (a.num_sms <= 0) return RQ_ECUDA;
+    return cuda_status(rq::launch_score(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+// rq_quant_inst.cuh -- instantiates the quantize / dequantize / sketch kernels
+// for one block size RQ_D and one dtype RQ_BF16 (set by the including file),
+// so that the heavy fully unrolled kernels compile in parallel units.
+#include "rq_quant_impl.cuh"
+
+namespace rq {
+
+template <int D, int PW, bool BF16, bool QJL>
+static cudaError_t launch_q(const QuantArgs &a, cudaStream_t st)
+{
+    auto kern = quantize_kernel<D, PW, BF16, QJL>;
+    const size_t smem = quantize_smem_bytes(D, QJL);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    constexpr int E = D < 128 ? D : 128;
+    const int64_t rows = a.nblocks * (D / E);
+    const int64_t tiles = (rows + kThreads - 1) / kThreads;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t cap = (int64_t)a.num_sms * (per_sm > 0 ? per_sm : 1);
+    const int64_t grid = tiles < cap ? tiles : cap;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
+        static_cast<const uint8_t *>(a.x), a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms,
+        a.m, static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
+    return cudaGetLastError();
+}
+
+template <int D, int PW, bool BF16>
+static cudaError_t launch_dq(const DequantArgs &a, cudaStream_t st)
+{
+    auto kern = dequantize_kernel<D, PW, BF16>;
+    const size_t smem = dequantize_smem_bytes(D);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    constexpr int E = D < 128 ? D : 128;
+    const int64_t rows = a.nblocks * (D / E);
+    const int64_t tiles = (rows + kThreads - 1) / kThreads;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t cap = (int64_t)a.num_sms * (per_sm > 0 ? per_sm : 1);
+    const int64_t grid = tiles < cap ? tiles : cap;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
+        static_cast<const uint8_t *>(a.codes), a.norms, a.nblocks, *a.tables, static_cast<uint8_t *>(a.out));
+    return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+static cudaError_t launch_sk(const SketchArgs &a, cudaStream_t st)
+{
+    auto kern = sketch_kernel<D, BF16>;
+    constexpr int E = D < 128 ? D : 128;
+    const size_t smem = (size_t)kThreads * E * 2;
+    const int64_t rows = a.nvec * (D / E);
+    const int64_t tiles = (rows + kThreads - 1) / kThreads;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t cap = (int64_t)a.num_sms * (per_sm > 0 ? per_sm : 1);
+    const int64_t grid = tiles < cap ? tiles : cap;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
+        static_cast<const uint8_t *>(a.x), a.nvec, a.m, static_cast<const uint16_t *>(a.proj), a.signs, a.norms);
+    return cudaGetLastError();
+}
+
+#define RQ_CAT2(a, b, c) a##_d##b##_##c
+#define RQ_CAT(a, b, c) RQ_CAT2(a, b, c)
+#if RQ_BF16
+#define RQ_DT bf16
+#else
+#define RQ_DT f16
+#endif
+
+cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_t st)
+{
+    const bool qjl = a.qsigns != nullptr;
+#define RQ_CASE(PW) \
+    case PW: return qjl ? launch_q<RQ_D, PW, RQ_BF16, true>(a, st) : launch_q<RQ_D, PW, RQ_BF16, false>(a, st);
+    switch (a.pw) {
+    RQ_CASE(1) RQ_CASE(2) RQ_CASE(3) RQ_CASE(4) RQ_CASE(5) RQ_CASE(6) RQ_CASE(7) RQ_CASE(8)
+    default: return cudaErrorInvalidValue;
+    }
+#undef RQ_CASE
+}
+
+cudaError_t RQ_CAT(launch_dequantize, RQ_D, RQ_DT)(const DequantArgs &a, cudaStream_t st)
+{
+#define RQ_CASE(PW) \
+    case PW: return launch_dq<RQ_D, PW, RQ_BF16>(a, st);
+    switch (a.pw) {
+    RQ_CASE(1) RQ_CASE(2) RQ_CASE(3) RQ_CASE(4) RQ_CASE(5) RQ_CASE(6) RQ_CASE(7) RQ_CASE(8)
+    default: return cudaErrorInvalidValue;
+    }
+#undef RQ_CASE
+}
+
+cudaError_t RQ_CAT(launch_sketch, RQ_D, RQ_DT)(const SketchArgs &a, cudaStream_t st)
+{
+    return launch_sk<RQ_D, RQ_BF16>(a, st);
+}
+
+}  // namespace rq

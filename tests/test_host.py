@@ -1,0 +1,132 @@
+"""Host-side checks of librq: the library loads, exports every entry point of
+include/rq.h, rejects bad arguments before touching the GPU, and its host
+tables (Lloyd-Max levels, storage sizes) agree with the oracle and the pages."""
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle as O
+from kv_quantization_b200 import _lib as L
+from tests.conftest import ROOT, read_golden
+
+HEADER = os.path.join(ROOT, "include", "rq.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(\w+)\s*\(", src, flags=re.M)) - {"if"})
+
+
+def test_header_and_binding_agree():
+    names = header_functions()
+    assert names == sorted(L.exported_symbols()), names
+
+
+def test_library_exports_every_header_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in header_functions():
+        assert name in exported, name
+    L.lib()  # loads
+
+
+def test_status_strings():
+    assert L.status_string(0) == "RQ_OK"
+    for s in (-1, -2, -3, -4, -5):
+        assert L.status_string(s).startswith("RQ_E")
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+def test_library_lloyd_max_equals_oracle(bits):
+    got = L.rq_lloyd_max(bits)
+    want = O.f32_table(bits)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_code_bytes():
+    assert L.rq_code_bytes(131072, 128, 4, L.RQ_CODES_INT8) == 131072
+    assert L.rq_code_bytes(4096 * 4096, 128, 3, L.RQ_CODES_PACKED) == 4096 * 4096 * 3 // 8
+    assert L.rq_code_bytes(4096 * 4096, 128, 5, L.RQ_CODES_PACKED) == 4096 * 4096 * 5 // 8
+    assert L.rq_code_bytes(100, 128, 4, L.RQ_CODES_PACKED) == -1
+    assert L.rq_code_bytes(128, 96, 4, L.RQ_CODES_PACKED) == -1
+
+
+def test_k_side_ratio_from_library_layout():
+    """Per-token bytes of a QJL key = m/8 sign bytes + one fp16 norm; the
+    ratio against bf16 keys reproduces the README's 7.53x / 14.22x / 3.88x."""
+    for hd, m, ratio in read_golden("qjl_k_side_ratio.txt"):
+        hd, m = int(hd), int(m)
+        per_token = m // 8 + np.dtype(np.float16).itemsize
+        assert round(hd * 2 / per_token, 2) == float(ratio)
+
+
+class FakeTensor:
+    """Stand-in device buffer: validation must fail before any dereference."""
+
+    def __init__(self, ptr, numel=1 << 20, dtype=None):
+        import torch
+        self._ptr, self._n = ptr, numel
+        self.dtype = dtype or torch.bfloat16
+
+    def data_ptr(self):
+        return self._ptr
+
+    def numel(self):
+        return self._n
+
+    def element_size(self):
+        return 2
+
+
+def _q(x, d=128, bits=4, layout=L.RQ_CODES_PACKED, cent=None, codes=None, norms=None, n=None):
+    cent = O.f32_table(bits) if cent is None else cent
+    codes = codes or FakeTensor(0x10000)
+    norms = norms or FakeTensor(0x20000)
+    L.rq_quantize(x, d, bits, layout, 1, 7, cent, codes, norms, stream=0, n=n)
+
+
+@pytest.mark.parametrize("case, status", [
+    (dict(d=96), -1), (dict(d=1024), -4), (dict(bits=9), -1), (dict(bits=0), -1), (dict(n=1000), -1),
+    (dict(layout=5), -1), (dict(cent=np.array([0.0, 0.0] + [1.0] * 14, np.float32)), -1),
+    (dict(cent=np.array([np.nan] * 16, np.float32)), -1),
+])
+def test_quantize_rejects_bad_arguments(case, status):
+    with pytest.raises(L.RQError) as e:
+        _q(FakeTensor(0x30000), **case)
+    assert e.value.status == status
+
+
+def test_quantize_rejects_null_and_misaligned():
+    with pytest.raises(L.RQError) as e:
+        _q(FakeTensor(0))
+    assert e.value.status == -1
+    with pytest.raises(L.RQError) as e:
+        _q(FakeTensor(0x30008))
+    assert e.value.status == -2
+
+
+def test_zero_length_is_a_noop():
+    _q(FakeTensor(0), n=0)    # nothing enqueued, nothing dereferenced
+
+
+def test_qjl_rejects_bad_m():
+    for m in (0, 4, 12, 520):
+        with pytest.raises(L.RQError) as e:
+            L.qjl_sketch(FakeTensor(0x40000), 128, m, FakeTensor(0x50000), FakeTensor(0x60000), FakeTensor(0x70000),
+                         stream=0)
+        assert e.value.status == -1
+    with pytest.raises(L.RQError):
+        L.qjl_make_projection(1, 256, 100, FakeTensor(0x50000), stream=0)
+
+
+def test_score_workspace_size_and_check():
+    assert L.qjl_score_workspace_bytes(8, 32, 256, 256) == 8 * 32 * 512 * 4
+    small = FakeTensor(0x90000, numel=16)
+    with pytest.raises(L.RQError) as e:
+        L.qjl_score(FakeTensor(0x40000), 8, 32, 256, 256, FakeTensor(0x50000), FakeTensor(0x60000),
+                    FakeTensor(0x70000), 1000, FakeTensor(0x80000), small, stream=0)
+    assert e.value.status == -3
