@@ -23,7 +23,8 @@
  *   - Pointers named x, codes, norms, out, proj, signs, scores, q and workspace
  *     are DEVICE pointers owned by the caller; `centroids` is a HOST pointer.
  *     The library keeps no pointer after a call returns, allocates no device
- *     memory and keeps no global state.
+ *     memory and keeps no global state besides one device error word
+ *     (rq_device_error).
  *   - Every call validates its arguments on the host, then enqueues its
  *     kernels asynchronously on `stream` (0 = legacy default stream) and
  *     returns.  Kernel faults surface at the caller's next synchronisation.
@@ -67,7 +68,8 @@ typedef enum {
     RQ_EALIGN = -2,        /* a device pointer is not 16-byte aligned */
     RQ_ESIZE = -3,         /* a size does not fit the kernels' index arithmetic */
     RQ_EUNSUPPORTED = -4,  /* valid but not implemented (d, bits, m, dtype combination) */
-    RQ_ECUDA = -5          /* a CUDA runtime call failed (launch error, ...) */
+    RQ_ECUDA = -5,         /* a CUDA runtime call failed (launch error, ...) */
+    RQ_EDEVICE = -6        /* a kernel's bounded wait expired (see rq_device_error) */
 } rq_status;
 
 typedef enum { RQ_F16 = 0, RQ_BF16 = 1 } rq_dtype;
@@ -75,6 +77,13 @@ typedef enum { RQ_CODES_PACKED = 0, RQ_CODES_INT8 = 1 } rq_layout;
 
 /* Human-readable name of a status code (static string). */
 const char *rq_status_string(int status);
+
+/* Device-side error word of the current device: RQ_EDEVICE if a kernel since
+ * the last clear gave up a bounded wait on the tensor core (its outputs are
+ * invalid; the kernel freed its resources and returned instead of hanging),
+ * else RQ_OK.  Synchronous (waits for the device); clear != 0 resets the word.
+ * Returns RQ_ECUDA if the word cannot be read. */
+rq_status rq_device_error(int clear);
 
 /* Bytes of code storage for n values in blocks of d: (n/d) * (d*bits/8) packed,
  * n for int8.  Returns -1 on invalid arguments. */

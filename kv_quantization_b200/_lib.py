@@ -42,6 +42,7 @@ def lib() -> C.CDLL:
             sig = {
                 "rq_status_string": (C.c_char_p, [i32]),
                 "rq_code_bytes": (i64, [i64, i32, i32, i32]),
+                "rq_device_error": (i32, [i32]),
                 "rq_lloyd_max": (i32, [i32, fp]),
                 "rq_quantize": (i32, [vp, i32, i64, i32, i32, i32, i32, u64, fp, vp, vp, vp]),
                 "rq_dequantize": (i32, [vp, vp, i64, i32, i32, i32, i32, u64, fp, vp, i32, vp]),
@@ -62,7 +63,7 @@ def lib() -> C.CDLL:
 
 def exported_symbols():
     """Names this binding expects librq.so to export."""
-    return ["rq_status_string", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
+    return ["rq_status_string", "rq_device_error", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
             "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score"]
 
 
@@ -104,6 +105,11 @@ def _dtype_code(t):
 
 def rq_code_bytes(n: int, d: int, bits: int, layout: int) -> int:
     return lib().rq_code_bytes(n, d, bits, layout)
+
+
+def rq_device_error(clear: bool = True) -> int:
+    """RQ_OK, or RQ_EDEVICE when a kernel gave up a bounded wait since the last clear."""
+    return lib().rq_device_error(int(clear))
 
 
 def rq_lloyd_max(bits: int) -> np.ndarray:

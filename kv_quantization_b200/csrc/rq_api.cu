@@ -16,6 +16,11 @@
 
 using rq::QuantTables;
 
+namespace rq {
+// Set (bitwise OR) by a kernel whose bounded wait on the tensor core expired.
+__device__ unsigned int g_device_error = 0;
+}  // namespace rq
+
 namespace {
 
 bool pow2_d(int d) { return d == 64 || d == 128 || d == 256 || d == 512; }
@@ -173,6 +178,7 @@ const char *rq_status_string(int status)
     case RQ_ESIZE: return "RQ_ESIZE: size out of range";
     case RQ_EUNSUPPORTED: return "RQ_EUNSUPPORTED: unsupported combination";
     case RQ_ECUDA: return "RQ_ECUDA: CUDA runtime error";
+    case RQ_EDEVICE: return "RQ_EDEVICE: a kernel gave up waiting on the tensor core; outputs are invalid";
     default: return "unknown rq_status";
     }
 }
@@ -313,6 +319,17 @@ rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m,
     a.norms = norms; a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
     return cuda_status(rq::launch_sketch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rq_status rq_device_error(int clear)
+{
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, rq::g_device_error, sizeof(word)) != cudaSuccess) return RQ_ECUDA;
+    if (clear && word) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(rq::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return RQ_ECUDA;
+    }
+    return word ? RQ_EDEVICE : RQ_OK;
 }
 
 size_t qjl_score_workspace_bytes(int64_t G, int n_q, int d, int m)

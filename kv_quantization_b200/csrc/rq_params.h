@@ -1,5 +1,6 @@
 // rq_params.h -- kernel parameter blocks of librq, shared by host and device code.
 #pragma once
+#include <cstddef>
 #include <cstdint>
 
 namespace rq {
@@ -9,6 +10,7 @@ namespace rq {
 constexpr float kLutMagic = 12582912.0f;
 constexpr int kMaxLutCells = 128;
 constexpr int kMaxLevels = 256;
+constexpr size_t kMaxSmemPerBlock = 232448;   // sm_100 opt-in limit (227 KB)
 
 // Per-call tables, passed by value as a kernel parameter (no device allocation).
 struct QuantTables {

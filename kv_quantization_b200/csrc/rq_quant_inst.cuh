@@ -2,6 +2,7 @@
 // for one block size RQ_D and one dtype RQ_BF16 (set by the including file),
 // so that the heavy fully unrolled kernels compile in parallel units.
 #include "rq_quant_impl.cuh"
+#include "rq_qjl_mma.cuh"
 
 namespace rq {
 
@@ -23,6 +24,25 @@ static cudaError_t launch_q(const QuantArgs &a, cudaStream_t st)
     kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
         static_cast<const uint8_t *>(a.x), a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms,
         a.m, static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
+    return cudaGetLastError();
+}
+
+// Tensor-core sketch path when S and the tiles fit in shared memory; returns
+// cudaErrorNotSupported when they do not (the caller then takes the SIMT path).
+template <int D, int PW, bool BF16, int MODE>
+static cudaError_t launch_mma(const QuantTables &T, const void *x, int64_t nvec, void *codes, uint16_t *norms,
+                              int m, const void *proj, uint8_t *signs, uint16_t *snorms, int num_sms, cudaStream_t st)
+{
+    const size_t smem = qjl_mma_smem_bytes(D, PW, m, T, MODE);
+    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+    auto kern = qjl_mma_kernel<D, PW, BF16, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (nvec + 127) / 128;
+    const int64_t grid = tiles < (int64_t)num_sms ? tiles : (int64_t)num_sms;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
+        static_cast<const uint8_t *>(x), nvec, T, static_cast<uint8_t *>(codes), norms, m,
+        static_cast<const uint16_t *>(proj), signs, snorms);
     return cudaGetLastError();
 }
 
@@ -75,8 +95,15 @@ static cudaError_t launch_sk(const SketchArgs &a, cudaStream_t st)
 cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_t st)
 {
     const bool qjl = a.qsigns != nullptr;
-#define RQ_CASE(PW) \
-    case PW: return qjl ? launch_q<RQ_D, PW, RQ_BF16, true>(a, st) : launch_q<RQ_D, PW, RQ_BF16, false>(a, st);
+#define RQ_CASE(PW)                                                                                       \
+    case PW:                                                                                              \
+        if (qjl) {                                                                                        \
+            cudaError_t e = launch_mma<RQ_D, PW, RQ_BF16, 0>(*a.tables, a.x, a.nblocks, a.codes, a.norms, a.m, \
+                                                             a.proj, a.qsigns, a.qnorms, a.num_sms, st);  \
+            if (e != cudaErrorNotSupported) return e;                                                     \
+            return launch_q<RQ_D, PW, RQ_BF16, true>(a, st);                                               \
+        }                                                                                                 \
+        return launch_q<RQ_D, PW, RQ_BF16, false>(a, st);
     switch (a.pw) {
     RQ_CASE(1) RQ_CASE(2) RQ_CASE(3) RQ_CASE(4) RQ_CASE(5) RQ_CASE(6) RQ_CASE(7) RQ_CASE(8)
     default: return cudaErrorInvalidValue;
@@ -97,6 +124,10 @@ cudaError_t RQ_CAT(launch_dequantize, RQ_D, RQ_DT)(const DequantArgs &a, cudaStr
 
 cudaError_t RQ_CAT(launch_sketch, RQ_D, RQ_DT)(const SketchArgs &a, cudaStream_t st)
 {
+    QuantTables T{};
+    cudaError_t e = launch_mma<RQ_D, 1, RQ_BF16, 1>(T, a.x, a.nvec, nullptr, nullptr, a.m, a.proj, a.signs, a.norms,
+                                                    a.num_sms, st);
+    if (e != cudaErrorNotSupported) return e;
     return launch_sk<RQ_D, RQ_BF16>(a, st);
 }
 

@@ -30,6 +30,14 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
+@pytest.fixture(autouse=True)
+def no_device_timeouts():
+    """Every kernel's bounded waits completed (no RQ_EDEVICE recorded)."""
+    yield
+    torch.cuda.synchronize()
+    assert L.rq_device_error(True) == 0
+
+
 def u16(t):
     return synth.as_u16(t).reshape(-1)
 
