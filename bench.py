@@ -42,11 +42,13 @@ WORKLOAD = "weight 4096x4096 bf16 student-t(4) std 0.02 + 0.1% outliers x20; d=1
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="rq", choices=["rq", "reference"])
     p.add_argument("--no-secondary", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--kernels-once", action="store_true",
+                   help="run each hot kernel once on inputs larger than L2 (profiling driver), print nothing else")
     return p.parse_args()
 
 
@@ -60,33 +62,39 @@ def peaks():
 
 
 class Clocks:
-    """nvidia-smi samples during the timed region."""
+    """nvidia-smi samples (every 20 ms) kept for the timed window only."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
-                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            time.sleep(0.5)        # let the sampler come up before the timed window
         except Exception:
             self.proc = None
-        return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
-    def __exit__(self, *a):
+    def window(self, t0, t1):
+        self.t0, self.t1 = t0, t1
+
+    def stop(self):
         if self.proc:
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -96,16 +104,18 @@ class Clocks:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [s.strip() for s in line.split(",")]
-            if len(parts) < 7:
+        for t, line in self.lines:
+            if self.t0 is not None and not (self.t0 <= t <= self.t1 + 0.05):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
             except ValueError:
                 continue
-            for name, v in zip(names, parts[3:7]):
+            for name, v in zip(names, parts[4:8]):
                 if v.lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
@@ -179,21 +189,28 @@ def run_device(args, rank, world):
 
     kern_ms = [[0.0] * n_ev for _ in range(args.steps)]
     step_ms = []
-    with Clocks(dev.index) as clk:
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-        torch.cuda.synchronize()
-        for s in range(args.steps):
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
-            step(evs)
-            torch.cuda.synchronize()
-            for k in range(n_ev):
-                kern_ms[s][k] = evs[k][0].elapsed_time(evs[k][1])
-            step_ms.append(sum(kern_ms[s]))
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
+    clk = Clocks(dev.index)
+    clk.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    evs_all = []
+    for s in range(args.steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+        step(evs)
+        evs_all.append(evs)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clk.window(t0, t1)
+    clk.stop()
+    for s, evs in enumerate(evs_all):
+        for k in range(n_ev):
+            kern_ms[s][k] = evs[k][0].elapsed_time(evs[k][1])
+        step_ms.append(sum(kern_ms[s]))
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
@@ -277,7 +294,7 @@ def e2e_measure(args, x, S, tabs, bufs, dev):
             "h2d_bytes_per_step": n * 2, "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 4)}
 
 
-def secondary_scores(dev):
+def secondary_scores(dev, reps=5):
     """QJL score tokens/s (key token-heads scored against all 32 queries per s)."""
     import torch
     import kv_quantization_b200 as rq
@@ -296,7 +313,7 @@ def secondary_scores(dev):
     out.append(_time_pair("kv 4x8x32768x128 QJL m=256",
                           lambda: rq.qjl_sketch(k, d, m, S, signs, kn),
                           lambda: rq.qjl_score(q, G, nq, d, m, S, signs, kn, T, scores, ws), G * T,
-                          2 * m * d * G * T, k.numel() * 2 + signs.numel() + kn.numel() * 2))
+                          2 * m * d * G * T, k.numel() * 2 + signs.numel() + kn.numel() * 2, reps))
     del k, signs, kn, scores, ws
     # TurboQuant-style 3-bit keys, head_dim 256: 2-bit + QJL m = d
     G, T, d, bits = 8, 131072, 256, 2
@@ -318,19 +335,20 @@ def secondary_scores(dev):
                           lambda: rq.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms,
                                                bits=bits, layout=rq.RQ_CODES_PACKED, use_signs=1, sign_seed=4,
                                                centroids=cent),
-                          G * T, 2 * m * d * G * T, k.numel() * 2 + codes.numel() + qs.numel() + 4 * G * T))
+                          G * T, 2 * m * d * G * T, k.numel() * 2 + codes.numel() + qs.numel() + 4 * G * T, reps))
     return out
 
 
-def _time_pair(name, prep, score, tokens, prep_flops, prep_bytes):
+def _time_pair(name, prep, score, tokens, prep_flops, prep_bytes, reps=5):
     import torch
     prep()
     score()
     torch.cuda.synchronize()
     res = {"workload": name}
+    if reps <= 1:
+        return res
     for label, fn in (("compress", prep), ("score", score)):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 5
         e0.record()
         for _ in range(reps):
             fn()
@@ -407,8 +425,39 @@ def run_reference(args):
             "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def kernels_once():
+    """Each hot kernel once, inputs larger than L2: 8192 x 8192 bf16 weight
+    (quantize, quantize+QJL, dequantize at 4 bits), the 4 x 8 x 32768 x 128 KV
+    cache (QJL sketch m=256 and its score), 131072 x 8 keys at head_dim 256
+    (2-bit + QJL m=d and its score)."""
+    import torch
+    import kv_quantization_b200 as rq
+    from kv_quantization_b200 import synth
+    dev = torch.device("cuda:0")
+    x = synth.student_t_outliers(8192, 8192, seed=1, device=dev).reshape(-1)
+    n, b = x.numel(), 4
+    cent = rq.rq_lloyd_max(b)
+    S = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    rq.qjl_make_projection(PROJ_SEED, M, D, S)
+    codes = torch.empty(rq.rq_code_bytes(n, D, b, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev)
+    norms = torch.empty(n // D, dtype=torch.int16, device=dev)
+    qs = torch.empty(n // D * M // 8, dtype=torch.uint8, device=dev)
+    qn = torch.empty(n // D, dtype=torch.int16, device=dev)
+    out = torch.empty_like(x)
+    rq.rq_quantize(x, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, cent, codes, norms)
+    rq.rq_quantize_qjl(x, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, cent, M, S, codes, norms, qs, qn)
+    rq.rq_dequantize(codes, norms, n, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, cent, out)
+    del x, out
+    secondary_scores(dev, reps=1)
+    torch.cuda.synchronize()
+    assert rq.rq_device_error(True) == 0
+
+
 def main():
     args = parse()
+    if args.kernels_once:
+        kernels_once()
+        return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     if args.impl == "reference":

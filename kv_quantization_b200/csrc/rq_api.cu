@@ -9,6 +9,8 @@
 #include <limits>
 #include <vector>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "rq.h"
@@ -154,6 +156,19 @@ rq_status make_tables(const float *centroids, int bits, int d, int use_signs, ui
 
 rq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ECUDA; }
 
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;   // driver entry point, looked up once
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
 // Lloyd-Max iteration for N(0,1): levels are conditional means of their cells,
 // thresholds are midpoints.  phi / Phi differences on the tail side.
 double npdf(double t) { return std::isinf(t) ? 0.0 : std::exp(-0.5 * t * t) * 0.39894228040143267794; }
@@ -166,6 +181,32 @@ double cell_mass(double a, double b)
 }
 
 }  // namespace
+
+bool rq::make_rows64_tmap(CUtensorMap *map, const void *ptr, int64_t rows)
+{
+    auto enc = tmap_encoder();
+    if (!enc || rows <= 0 || rows >= ((int64_t)1 << 31)) return false;
+    const cuuint64_t dims[2] = {64, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {64, 256};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool rq::make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d)
+{
+    auto enc = tmap_encoder();
+    if (!enc || n <= 0 || n >= ((int64_t)1 << 31) || d % 64) return false;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)(d / 64), (cuuint64_t)n};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)d * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 extern "C" {
 
@@ -224,7 +265,7 @@ static rq_status check_common(int64_t n, int d, int bits, rq_layout layout)
     if (bits < 1 || bits > 8) return RQ_EINVAL;
     if (layout != RQ_CODES_PACKED && layout != RQ_CODES_INT8) return RQ_EINVAL;
     if (n < 0 || n % d) return RQ_EINVAL;
-    if (n > ((int64_t)1 << 40)) return RQ_ESIZE;
+    if (n / 64 >= ((int64_t)1 << 31)) return RQ_ESIZE;   // TMA row coordinates are int32
     return RQ_OK;
 }
 
@@ -251,6 +292,7 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
     a.m = qjl ? m : 0; a.proj = proj; a.qsigns = qjl_signs; a.qnorms = qjl_norms;
     a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
+    if (!rq::make_rows64_tmap(&a.tmap_x, x, n / 64)) return RQ_ECUDA;
     return cuda_status(rq::launch_quantize(a, stream));
 }
 
@@ -290,6 +332,7 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
     a.bf16 = out_dtype == RQ_BF16; a.tables = &T; a.out = out;
     a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
+    if (!rq::make_rows64_tmap(&a.tmap_out, out, n / 64)) return RQ_ECUDA;
     return cuda_status(rq::launch_dequantize(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -318,6 +361,7 @@ rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m,
     a.x = x; a.nvec = n_vec; a.d = d; a.m = m; a.bf16 = dtype == RQ_BF16; a.proj = proj; a.signs = signs;
     a.norms = norms; a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
+    a.has_tmap_k = rq::make_vectors_tmap(&a.tmap_k, x, n_vec, d);
     return cuda_status(rq::launch_sketch(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "rq_params.h"
@@ -21,6 +22,7 @@ struct QuantArgs {
     uint8_t *qsigns;
     uint16_t *qnorms;
     int num_sms;
+    CUtensorMap tmap_x;        // input as [n/64][64] 16-bit rows, 256-row boxes, 128-byte swizzle
 };
 
 struct DequantArgs {
@@ -32,6 +34,7 @@ struct DequantArgs {
     const QuantTables *tables;
     void *out;
     int num_sms;
+    CUtensorMap tmap_out;      // output as [n/64][64] 16-bit rows, 256-row boxes, 128-byte swizzle
 };
 
 struct SketchArgs {
@@ -43,6 +46,8 @@ struct SketchArgs {
     uint8_t *signs;
     uint16_t *norms;
     int num_sms;
+    CUtensorMap tmap_k;        // keys as {64, d/64, n_vec} 16-bit, {64, 1, 128} boxes, 128-byte swizzle
+    bool has_tmap_k;
 };
 
 struct ScoreArgs {
@@ -70,6 +75,12 @@ cudaError_t launch_sketch(const SketchArgs &a, cudaStream_t st);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t st);
 size_t score_workspace_bytes(int64_t G, int nq, int d, int m);
 size_t quantize_smem_bytes(int d, bool qjl);
+// Encode the [rows][64] 16-bit row view of `ptr` as a TMA map (256-row boxes,
+// 128-byte swizzle); false if the driver refuses it.
+bool make_rows64_tmap(CUtensorMap *map, const void *ptr, int64_t rows);
+// Encode vectors[n][d] (16-bit) as {64, d/64, n} with {64, 1, 128} boxes:
+// one box is one 64-column region of 128 vectors, the tensor-core A layout.
+bool make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d);
 size_t dequantize_smem_bytes(int d);
 
 }  // namespace rq

@@ -1,0 +1,408 @@
+// rq_qjl_v2.cuh -- pipelined QJL sketch kernels for d = 128 (sm_100a).
+//
+// MODE 0 (rq_quantize_qjl): 256 threads quantize a 128-block tile exactly as
+//   quantize_v2_kernel (TMA input ring, 64 values per thread), rebuild the
+//   fp32 reconstruction, form the residual r = x - x^32 and write bf16(r) into
+//   a double-buffered 128 x 128 A tile (128-byte swizzled, K-major); one
+//   thread issues the tcgen05 MMAs of tile i into TMEM accumulator i mod 2
+//   while the threads already work on tile i+1; the sign-packing epilogue of
+//   tile i runs when tile i+2 needs its A buffer back.
+// MODE 1 (qjl_sketch): 3-D TMA loads put 128 keys straight into the A layout
+//   (one 64-column region per load); the threads only compute the canonical
+//   fp32 norms from shared memory; MMA of tile i overlaps the norm pass of
+//   tile i+1 and the epilogue of tile i-1.
+//
+// Epilogue: 8 warps; warp w reads TMEM lanes 32 (w mod 4) .. +31 (its 32
+// vectors) and every other 32-column chunk starting at chunk w / 4, packs the
+// 32 sign bits of a chunk into one word (bit i = P_i >= 0) and stores it.
+#pragma once
+#include "rq_qjl_mma.cuh"
+#include "rq_v2.cuh"
+
+namespace rq {
+
+constexpr int kQ2Stages = 3;
+
+__host__ __device__ inline uint32_t qjl_v2_tmem_cols(int m)
+{
+    uint32_t c = 32;
+    while (c < 2u * (uint32_t)qjl_mma_m16(m)) c <<= 1;
+    return c;
+}
+
+// Shared memory (bytes, with 1024-byte alignment slack).
+__host__ __device__ inline size_t qjl_v2_smem(int mode, int pw, int m, const QuantTables &T, int stages)
+{
+    const size_t S = (size_t)qjl_mma_m16(m) * 128 * 2;            // m16 rows x 128 bf16, 2 regions
+    size_t b = 1024 + S;
+    if (mode == 0) {
+        b += (size_t)stages * kTileBytes2;                        // input ring
+        b += 2 * (size_t)128 * 128 * 2;                           // A double buffer
+        b += lut_bytes_v2(T) + ((size_t)1 << pw) * 32 * 4 + 64 * 4;
+    } else {
+        b += (size_t)stages * 128 * 128 * 2;                      // A ring (TMA targets)
+    }
+    return b + 8 * (stages + 2) + 16;
+}
+
+// Sign-pack epilogue of one 128-vector tile from TMEM accumulator columns
+// [col0, col0 + m16).
+__device__ __forceinline__ void qjl_v2_epilogue(uint32_t tmem, uint32_t col0, int m, int m16, int64_t tok0,
+                                                int64_t nvec, uint8_t *__restrict__ signs, bool ok)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tok = tok0 + (warp & 3) * 32 + lane;
+    const bool tv = ok && tok < nvec;
+    uint8_t *dst = signs + tok * (m / 8);
+    for (int c0 = (warp >> 2) * 32; c0 < m16; c0 += 64) {
+        uint32_t acc[32];
+        tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + col0 + (uint32_t)c0, acc);
+        tmem_ld_wait();
+        uint32_t word = 0u;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) word |= (__uint_as_float(acc[i]) >= 0.0f ? 1u : 0u) << i;
+        if (tv && c0 < m) {
+            const int nb = min(4, (m - c0) / 8);
+            if (nb == 4 && (m & 31) == 0) {
+                *reinterpret_cast<uint32_t *>(dst + c0 / 8) = word;
+            } else {
+                for (int b = 0; b < nb; ++b) dst[c0 / 8 + b] = (uint8_t)(word >> (8 * b));
+            }
+        }
+    }
+}
+
+// One thread issues the MMAs of a 128 x m16 x 128 tile: A (2 regions of 128
+// rows) x S^T (2 regions of m16 rows), into TMEM columns [col0, col0 + m16).
+__device__ __forceinline__ void qjl_v2_issue(uint32_t sA, uint32_t sS, int m16, uint32_t tmem_col)
+{
+#pragma unroll
+    for (int kc = 0; kc < 2; ++kc) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint64_t adesc = sdesc_k_sw128(sA + (uint32_t)kc * 16384u + (uint32_t)k * 32u);
+            for (int n0 = 0; n0 < m16; n0 += 256) {
+                const int N = min(256, m16 - n0);
+                const uint64_t bdesc =
+                    sdesc_k_sw128(sS + (uint32_t)kc * (uint32_t)m16 * 128u + (uint32_t)n0 * 128u + (uint32_t)k * 32u);
+                mma_f16(tmem_col + (uint32_t)n0, adesc, bdesc, idesc_f16(true, 128, N), (kc | k) != 0);
+            }
+        }
+    }
+}
+
+template <bool SBF16>
+__device__ __forceinline__ void stage_projection(const uint16_t *__restrict__ proj, uint8_t *s_S, int m, int m16)
+{
+    for (int idx = threadIdx.x; idx < m16 * 16; idx += blockDim.x) {
+        const int i = idx >> 4, c = idx & 15;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i < m) v = __ldg(reinterpret_cast<const uint4 *>(proj + (size_t)i * 128) + c);
+        *reinterpret_cast<uint4 *>(s_S + (size_t)(c >> 3) * m16 * 128 + sw128_offset(i, c & 7)) = v;
+    }
+}
+
+// -------------------------------------------------------------- MODE 0
+
+template <int PW, bool BF16, int STAGES>
+__global__ void __launch_bounds__(kT2, 1)
+qjl_v2_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, const __grid_constant__ QuantTables T,
+                    uint8_t *__restrict__ codes, uint16_t *__restrict__ norms, int m,
+                    const uint16_t *__restrict__ proj, uint8_t *__restrict__ qsigns, uint16_t *__restrict__ qnorms)
+{
+    constexpr int D = 128, TPB = 2;
+    constexpr int CB = kE2 * PW / 8;
+    constexpr int NW = kE2 * PW / 32;
+    const int m16 = qjl_mma_m16(m);
+    const uint32_t ncols = qjl_v2_tmem_cols(m);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *s_S = base;
+    uint8_t *ring = s_S + (size_t)m16 * 256;
+    uint8_t *s_A = ring + (size_t)STAGES * kTileBytes2;             // 2 x 32 KB
+    uint8_t *lutb = s_A + 2 * 32768;
+    float *bnd = reinterpret_cast<float *>(lutb);
+    float *cent = reinterpret_cast<float *>(lutb + lut_bytes_v2(T));
+    uint32_t *pmask = reinterpret_cast<uint32_t *>(cent + (1 << PW) * 32);
+    uint64_t *full = reinterpret_cast<uint64_t *>(pmask + 64);
+    uint64_t *mma_bar = full + STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, part = tid & 1;
+    const int64_t nrows = nblocks * TPB;
+    const int64_t ntiles = (nrows + kT2 - 1) / kT2;
+    if (tid == 0) {
+        prefetch_tmap(&tmx);
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        mbar_init(&mma_bar[0], 1);
+        mbar_init(&mma_bar[1], 1);
+        fence_barrier_init();
+        for (int s = 0; s < STAGES; ++s) {
+            const int64_t t = blockIdx.x + (int64_t)s * gridDim.x;
+            if (t < ntiles) {
+                mbar_arrive_expect_tx(&full[s], kTileBytes2);
+                tma_load_2d(ring + s * kTileBytes2, &tmx, 0, (int)(t * kT2), &full[s]);
+            }
+        }
+    }
+    stage_projection<true>(proj, s_S, m, m16);
+    setup_lut_v2(T, reinterpret_cast<uint2 *>(lutb), bnd);
+    for (int i = tid; i < (1 << PW) * 32; i += kT2) {
+        const int k = i >> 5;
+        cent[i] = k < T.levels ? T.centroid[k] : 0.0f;
+    }
+    setup_pair_masks(T, pmask, D);
+    if (warp == 0) tmem_alloc(tmem_slot, ncols);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t sS = smem_u32(s_S), sA0 = smem_u32(s_A);
+
+    const float2 la = make_float2(T.lut_a, T.lut_a), lb = make_float2(T.lut_b, T.lut_b);
+    const int cells = T.lut_cells, levels = T.levels;
+    const uint32_t cells_m1 = (uint32_t)(cells > 0 ? cells - 1 : 0);
+    const uint8_t *lut_lane = lutb + (lane & 15) * 8;
+    const float *cent_lane = cent + lane;
+    const uint4 *pmv = reinterpret_cast<const uint4 *>(pmask + part * 32);
+    bool ok = true;
+    uint32_t mma_phase[2] = {0u, 0u};
+    int64_t i = 0;
+
+    for (;; ++i) {
+        const int64_t t = blockIdx.x + i * gridDim.x;
+        if (t >= ntiles) break;
+        const int s = (int)(i % STAGES);
+        const bool got = mbar_wait(&full[s], (uint32_t)((i / STAGES) & 1));
+        if (__syncthreads_or(!got)) { ok = false; break; }
+        uint8_t *tile = ring + s * kTileBytes2;
+        uint32_t u[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint4 v = *sw_row_chunk(tile, tid, k);
+            const uint4 q = pmv[k];
+            u[4 * k] = v.x ^ q.x; u[4 * k + 1] = v.y ^ q.y; u[4 * k + 2] = v.z ^ q.z; u[4 * k + 3] = v.w ^ q.w;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t tn = t + (int64_t)STAGES * gridDim.x;
+            if (tn < ntiles) {
+                mbar_arrive_expect_tx(&full[s], kTileBytes2);
+                tma_load_2d(tile, &tmx, 0, (int)(tn * kT2), &full[s]);
+            }
+        }
+        const int64_t row = t * kT2 + tid;
+        const bool valid = row < nrows;
+
+        // ---- quantize (canonical; as quantize_v2_kernel)
+        float2 P[32];
+        row_to_pairs<BF16>(u, P);
+        const float n32 = __fsqrt_rn(combine_parts<TPB>(row_sumsq(P)));
+        fwht_row<TPB>(P, part);
+        const float inv = n32 > 0.0f ? __frcp_rn(n32) : 0.0f;
+        const float2 inv2 = make_float2(inv, inv);
+        uint32_t w[NW];
+#pragma unroll
+        for (int k = 0; k < NW; ++k) w[k] = 0u;
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) {
+            const float2 y = __fmul2_rn(P[i2], inv2);
+            uint32_t c0, c1;
+            if (cells > 0) {
+                const float2 f = __ffma2_rn(y, la, lb);
+                c0 = lut_code_v2(y.x, f.x, lut_lane, cells_m1);
+                c1 = lut_code_v2(y.y, f.y, lut_lane, cells_m1);
+            } else {
+                c0 = bsearch_code(y.x, bnd, levels);
+                c1 = bsearch_code(y.y, bnd, levels);
+            }
+            const int b0 = i2 * PW, b1 = (i2 + 32) * PW;
+            w[b0 >> 5] |= c0 << (b0 & 31);
+            if ((b0 & 31) + PW > 32) w[(b0 >> 5) + 1] |= c0 >> (32 - (b0 & 31));
+            w[b1 >> 5] |= c1 << (b1 & 31);
+            if ((b1 & 31) + PW > 32) w[(b1 >> 5) + 1] |= c1 >> (32 - (b1 & 31));
+        }
+        const uint16_t n16 = norm_to_h16(n32);
+        if (valid) {
+            store_bytes<CB>(codes + row * CB, w);
+            if (part == 0) norms[row / TPB] = n16;
+        }
+
+        // ---- residual r' = s*x - w*scale (fp32, canonical), r = s * r'
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) {
+            P[i2].x = cent_lane[unpack_code<kE2, PW>(w, i2) * 32];
+            P[i2].y = cent_lane[unpack_code<kE2, PW>(w, i2 + 32) * 32];
+        }
+        fwht_row<TPB>(P, part);
+        const float nsc = -__fmul_rn(h16_to_f32(n16), 1.0f / (float)D);
+        const float2 nsc2 = make_float2(nsc, nsc);
+        float2 X[32];
+        row_to_pairs<BF16>(u, X);
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) P[i2] = __fadd2_rn(X[i2], __fmul2_rn(P[i2], nsc2));
+        const float rn32 = __fsqrt_rn(combine_parts<TPB>(row_sumsq(P)));
+        if (valid && part == 0) qnorms[row / TPB] = norm_to_h16(rn32);
+
+        // ---- A buffer a = i mod 2: tile i-2's MMA must be done; drain its accumulator
+        const int a = (int)(i & 1);
+        if (i >= 2) {
+            if (ok && !mbar_wait(&mma_bar[a], mma_phase[a])) ok = false;
+            mma_phase[a] ^= 1u;
+            tc_fence_after();
+            qjl_v2_epilogue(tmem, (uint32_t)(a * m16), m, m16, (t - 2 * (int64_t)gridDim.x) * 128, nblocks, qsigns, ok);
+            tc_fence_before();
+        }
+        uint8_t *A = s_A + a * 32768;
+        const int arow = tid >> 1;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int wd = 4 * k + q;
+                const float va = wd < 16 ? P[2 * wd].x : P[2 * wd - 32].y;
+                const float vb = wd < 16 ? P[2 * wd + 1].x : P[2 * wd - 31].y;
+                o[q] = pack2<true>(va, vb);
+            }
+            const uint4 q = pmv[k];
+            *reinterpret_cast<uint4 *>(A + part * 16384 + sw128_offset(arow, k)) =
+                make_uint4(o[0] ^ q.x, o[1] ^ q.y, o[2] ^ q.z, o[3] ^ q.w);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+        if (tid == 0) {
+            tc_fence_after();
+            qjl_v2_issue(sA0 + (uint32_t)a * 32768u, sS, m16, tmem + (uint32_t)(a * m16));
+            mma_commit(&mma_bar[a]);
+        }
+    }
+    // drain the last two tiles (i = number of tiles this CTA processed)
+    for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j) {
+        const int a = (int)(j & 1);
+        if (ok && !mbar_wait(&mma_bar[a], mma_phase[a])) ok = false;
+        mma_phase[a] ^= 1u;
+        tc_fence_after();
+        qjl_v2_epilogue(tmem, (uint32_t)(a * m16), m, m16, (blockIdx.x + j * (int64_t)gridDim.x) * 128, nblocks, qsigns,
+                        ok);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+// -------------------------------------------------------------- MODE 1
+
+// 3-D view of the keys: {64 values, 2 chunks, n tokens}; box {64, 1, 128}.
+template <bool BF16, int STAGES>
+__global__ void __launch_bounds__(kT2, 1)
+qjl_v2_sketch_kernel(const __grid_constant__ CUtensorMap tmk, int64_t nvec, int m, const uint16_t *__restrict__ proj,
+                     uint8_t *__restrict__ signs, uint16_t *__restrict__ norms)
+{
+    constexpr int ATILE = 128 * 128 * 2;
+    const int m16 = qjl_mma_m16(m);
+    const uint32_t ncols = qjl_v2_tmem_cols(m);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *s_S = base;
+    uint8_t *ring = s_S + (size_t)m16 * 256;
+    uint64_t *full = reinterpret_cast<uint64_t *>(ring + (size_t)STAGES * ATILE);
+    uint64_t *mma_bar = full + STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, part = tid & 1;
+    const int64_t ntiles = (nvec + 127) / 128;
+    if (tid == 0) {
+        prefetch_tmap(&tmk);
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        mbar_init(&mma_bar[0], 1);
+        mbar_init(&mma_bar[1], 1);
+        fence_barrier_init();
+        for (int s = 0; s < STAGES; ++s) {
+            const int64_t t = blockIdx.x + (int64_t)s * gridDim.x;
+            if (t < ntiles) {
+                mbar_arrive_expect_tx(&full[s], ATILE);
+                tma_load_3d(ring + s * ATILE, &tmk, 0, 0, (int)(t * 128), &full[s]);
+                tma_load_3d(ring + s * ATILE + 16384, &tmk, 0, 1, (int)(t * 128), &full[s]);
+            }
+        }
+    }
+    stage_projection<BF16>(proj, s_S, m, m16);
+    if (warp == 0) tmem_alloc(tmem_slot, ncols);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t sS = smem_u32(s_S), sR = smem_u32(ring);
+    bool ok = true;
+    uint32_t mma_phase[2] = {0u, 0u};
+    int64_t i = 0;
+
+    for (;; ++i) {
+        const int64_t t = blockIdx.x + i * gridDim.x;
+        if (t >= ntiles) break;
+        const int s = (int)(i % STAGES);
+        const bool got = mbar_wait(&full[s], (uint32_t)((i / STAGES) & 1));
+        if (__syncthreads_or(!got)) { ok = false; break; }
+        // MMA of tile i as soon as its keys have landed
+        if (tid == 0) {
+            tc_fence_after();
+            qjl_v2_issue(sR + (uint32_t)s * ATILE, sS, m16, tmem + (uint32_t)((i & 1) * m16));
+            mma_commit(&mma_bar[i & 1]);
+        }
+        // canonical fp32 norm of each key: thread = (key tid/2, half tid%2)
+        {
+            const uint8_t *Ar = ring + s * ATILE + part * 16384;
+            const int r = tid >> 1;
+            uint32_t u[32];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(Ar + sw128_offset(r, k));
+                u[4 * k] = v.x; u[4 * k + 1] = v.y; u[4 * k + 2] = v.z; u[4 * k + 3] = v.w;
+            }
+            float2 P[32];
+            row_to_pairs<BF16>(u, P);
+            const float n32 = __fsqrt_rn(combine_parts<2>(row_sumsq(P)));
+            const int64_t tok = t * 128 + r;
+            if (part == 0 && tok < nvec) norms[tok] = norm_to_h16(n32);
+        }
+        // tile i-1: accumulator ready -> signs; its A stage returns to the TMA ring
+        if (i >= 1) {
+            const int a = (int)((i - 1) & 1);
+            if (ok && !mbar_wait(&mma_bar[a], mma_phase[a])) ok = false;
+            mma_phase[a] ^= 1u;
+            tc_fence_after();
+            const int64_t tp = t - gridDim.x;
+            qjl_v2_epilogue(tmem, (uint32_t)(a * m16), m, m16, tp * 128, nvec, signs, ok);
+            tc_fence_before();
+            if (tid == 0) {
+                const int sp = (int)((i - 1) % STAGES);
+                const int64_t tn = tp + (int64_t)STAGES * gridDim.x;
+                if (tn < ntiles) {
+                    mbar_arrive_expect_tx(&full[sp], ATILE);
+                    tma_load_3d(ring + sp * ATILE, &tmk, 0, 0, (int)(tn * 128), &full[sp]);
+                    tma_load_3d(ring + sp * ATILE + 16384, &tmk, 0, 1, (int)(tn * 128), &full[sp]);
+                }
+            }
+        }
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+    }
+    if (i >= 1) {
+        const int a = (int)((i - 1) & 1);
+        if (ok && !mbar_wait(&mma_bar[a], mma_phase[a])) ok = false;
+        mma_phase[a] ^= 1u;
+        tc_fence_after();
+        qjl_v2_epilogue(tmem, (uint32_t)(a * m16), m, m16, (blockIdx.x + (i - 1) * (int64_t)gridDim.x) * 128, nvec,
+                        signs, ok);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+}  // namespace rq

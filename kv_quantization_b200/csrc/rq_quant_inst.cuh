@@ -3,6 +3,8 @@
 // so that the heavy fully unrolled kernels compile in parallel units.
 #include "rq_quant_impl.cuh"
 #include "rq_qjl_mma.cuh"
+#include "rq_v2.cuh"
+#include "rq_qjl_v2.cuh"
 
 namespace rq {
 
@@ -46,23 +48,88 @@ static cudaError_t launch_mma(const QuantTables &T, const void *x, int64_t nvec,
     return cudaGetLastError();
 }
 
-template <int D, int PW, bool BF16>
-static cudaError_t launch_dq(const DequantArgs &a, cudaStream_t st)
+// Pipelined tensor-core paths for d = 128 (rq_qjl_v2.cuh); NotSupported when
+// the shape or the shared memory does not fit.
+template <int PW, bool BF16>
+static cudaError_t launch_qjl_v2(const QuantArgs &a, cudaStream_t st)
 {
-    auto kern = dequantize_kernel<D, PW, BF16>;
-    const size_t smem = dequantize_smem_bytes(D);
+    const QuantTables &T = *a.tables;
+    const int64_t tiles = (a.nblocks + 127) / 128;
+    const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
+    if (2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
+    size_t smem = qjl_v2_smem(0, PW, a.m, T, 3);
+    if (smem <= kMaxSmemPerBlock) {
+        auto kern = qjl_v2_quant_kernel<PW, BF16, 3>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_x, a.nblocks, T, static_cast<uint8_t *>(a.codes),
+                                                                a.norms, a.m, static_cast<const uint16_t *>(a.proj),
+                                                                a.qsigns, a.qnorms);
+        return cudaGetLastError();
+    }
+    smem = qjl_v2_smem(0, PW, a.m, T, 2);
+    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+    auto kern = qjl_v2_quant_kernel<PW, BF16, 2>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    constexpr int E = D < 128 ? D : 128;
-    const int64_t rows = a.nblocks * (D / E);
-    const int64_t tiles = (rows + kThreads - 1) / kThreads;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_x, a.nblocks, T, static_cast<uint8_t *>(a.codes),
+                                                            a.norms, a.m, static_cast<const uint16_t *>(a.proj),
+                                                            a.qsigns, a.qnorms);
+    return cudaGetLastError();
+}
+
+template <bool BF16>
+static cudaError_t launch_sketch_v2(const SketchArgs &a, cudaStream_t st)
+{
+    if (!a.has_tmap_k || 2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
+    QuantTables T{};
+    const size_t smem = qjl_v2_smem(1, 1, a.m, T, 3);
+    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+    auto kern = qjl_v2_sketch_kernel<BF16, 3>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (a.nvec + 127) / 128;
+    const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_k, a.nvec, a.m,
+                                                            static_cast<const uint16_t *>(a.proj), a.signs, a.norms);
+    return cudaGetLastError();
+}
+
+template <int D, int PW, bool BF16>
+static cudaError_t launch_q2(const QuantArgs &a, cudaStream_t st)
+{
+    auto kern = quantize_v2_kernel<D, PW, BF16>;
+    const size_t smem = quantize_v2_smem(D, *a.tables);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = a.nblocks * (D / kE2);
+    const int64_t tiles = (rows + kT2 - 1) / kT2;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kT2, smem);
     if (e != cudaSuccess) return e;
     const int64_t cap = (int64_t)a.num_sms * (per_sm > 0 ? per_sm : 1);
     const int64_t grid = tiles < cap ? tiles : cap;
-    kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
-        static_cast<const uint8_t *>(a.codes), a.norms, a.nblocks, *a.tables, static_cast<uint8_t *>(a.out));
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_x, rows, *a.tables,
+                                                            static_cast<uint8_t *>(a.codes), a.norms);
+    return cudaGetLastError();
+}
+
+template <int D, int PW, bool BF16>
+static cudaError_t launch_dq2(const DequantArgs &a, cudaStream_t st)
+{
+    auto kern = dequantize_v2_kernel<D, PW, BF16>;
+    const size_t smem = dequantize_v2_smem(D, PW);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = a.nblocks * (D / kE2);
+    const int64_t tiles = (rows + kT2 - 1) / kT2;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kT2, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t cap = (int64_t)a.num_sms * (per_sm > 0 ? per_sm : 1);
+    const int64_t grid = tiles < cap ? tiles : cap;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(static_cast<const uint8_t *>(a.codes), a.norms, rows,
+                                                            *a.tables, a.tmap_out);
     return cudaGetLastError();
 }
 
@@ -98,12 +165,16 @@ cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_
 #define RQ_CASE(PW)                                                                                       \
     case PW:                                                                                              \
         if (qjl) {                                                                                        \
+            if (RQ_D == 128) {                                                                            \
+                cudaError_t e2 = launch_qjl_v2<PW, RQ_BF16>(a, st);                                       \
+                if (e2 != cudaErrorNotSupported) return e2;                                               \
+            }                                                                                             \
             cudaError_t e = launch_mma<RQ_D, PW, RQ_BF16, 0>(*a.tables, a.x, a.nblocks, a.codes, a.norms, a.m, \
                                                              a.proj, a.qsigns, a.qnorms, a.num_sms, st);  \
             if (e != cudaErrorNotSupported) return e;                                                     \
             return launch_q<RQ_D, PW, RQ_BF16, true>(a, st);                                               \
         }                                                                                                 \
-        return launch_q<RQ_D, PW, RQ_BF16, false>(a, st);
+        return launch_q2<RQ_D, PW, RQ_BF16>(a, st);
     switch (a.pw) {
     RQ_CASE(1) RQ_CASE(2) RQ_CASE(3) RQ_CASE(4) RQ_CASE(5) RQ_CASE(6) RQ_CASE(7) RQ_CASE(8)
     default: return cudaErrorInvalidValue;
@@ -114,7 +185,7 @@ cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_
 cudaError_t RQ_CAT(launch_dequantize, RQ_D, RQ_DT)(const DequantArgs &a, cudaStream_t st)
 {
 #define RQ_CASE(PW) \
-    case PW: return launch_dq<RQ_D, PW, RQ_BF16>(a, st);
+    case PW: return launch_dq2<RQ_D, PW, RQ_BF16>(a, st);
     switch (a.pw) {
     RQ_CASE(1) RQ_CASE(2) RQ_CASE(3) RQ_CASE(4) RQ_CASE(5) RQ_CASE(6) RQ_CASE(7) RQ_CASE(8)
     default: return cudaErrorInvalidValue;
@@ -124,6 +195,10 @@ cudaError_t RQ_CAT(launch_dequantize, RQ_D, RQ_DT)(const DequantArgs &a, cudaStr
 
 cudaError_t RQ_CAT(launch_sketch, RQ_D, RQ_DT)(const SketchArgs &a, cudaStream_t st)
 {
+    if (RQ_D == 128) {
+        cudaError_t e2 = launch_sketch_v2<RQ_BF16>(a, st);
+        if (e2 != cudaErrorNotSupported) return e2;
+    }
     QuantTables T{};
     cudaError_t e = launch_mma<RQ_D, 1, RQ_BF16, 1>(T, a.x, a.nvec, nullptr, nullptr, a.m, a.proj, a.signs, a.norms,
                                                     a.num_sms, st);
