@@ -11,6 +11,7 @@
 
 #include "rq_common.cuh"
 #include "rq_kernels.h"
+#include "qjl_score_v3.cuh"
 
 namespace rq {
 
@@ -162,7 +163,37 @@ score_kernel(const float *__restrict__ ws, int nq, int d, int m, const uint8_t *
 
 size_t score_workspace_bytes(int64_t G, int nq, int d, int m)
 {
-    return (size_t)G * (size_t)nq * (size_t)(d + m) * sizeof(float);
+    const size_t v1 = (size_t)G * (size_t)nq * (size_t)(d + m) * sizeof(float);
+    const size_t v2 = sc2_ws_bytes(G, nq, d, m, true);
+    return v1 > v2 ? v1 : v2;
+}
+
+// Tensor-core score path; cudaErrorNotSupported when the shape does not fit.
+template <int PW, bool TWO>
+static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
+{
+    if (a.nq > 128) return cudaErrorNotSupported;
+    const size_t smem = sc3_smem(a.nq, a.d, a.m, TWO, PW);
+    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+    uint16_t *wsB = reinterpret_cast<uint16_t *>(a.workspace);
+    const size_t rows = (size_t)a.G * a.nq;
+    float *wsN = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.workspace) +
+                                           ((rows * sc2_kb(a.d, a.m, TWO) * 2 + 255) & ~(size_t)255));
+    const size_t psmem = ((size_t)2 * kSc2PrologueQ * a.d + kSc2PrologueQ) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(score_v2_prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    if (e != cudaSuccess) return e;
+    score_v2_prologue<<<dim3((unsigned)a.G, (unsigned)((a.nq + kSc2PrologueQ - 1) / kSc2PrologueQ)), 256, psmem, st>>>(
+        a.q, a.nq, a.d, a.m, static_cast<const uint16_t *>(a.proj), a.proj_bf16, *a.tables, TWO, wsB, wsN);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    auto kern = score_v3_kernel<PW, TWO>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t items = a.G * ((a.T + 127) / 128);
+    const int64_t grid = items < (int64_t)a.num_sms ? items : (int64_t)a.num_sms;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kSc3Threads, smem, st>>>(wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms,
+                                                                     a.T, a.G, a.codes, a.norms, *a.tables, a.scores);
+    return cudaGetLastError();
 }
 
 template <int PW, bool TWO>
@@ -182,6 +213,25 @@ static cudaError_t launch_score_main(const ScoreArgs &a, cudaStream_t st)
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t st)
 {
     const bool two = a.codes != nullptr;
+    {
+        cudaError_t e2 = cudaErrorNotSupported;
+        if (!two) {
+            e2 = launch_score_v2<1, false>(a, st);
+        } else {
+            switch (a.pw) {
+            case 1: e2 = launch_score_v2<1, true>(a, st); break;
+            case 2: e2 = launch_score_v2<2, true>(a, st); break;
+            case 3: e2 = launch_score_v2<3, true>(a, st); break;
+            case 4: e2 = launch_score_v2<4, true>(a, st); break;
+            case 5: e2 = launch_score_v2<5, true>(a, st); break;
+            case 6: e2 = launch_score_v2<6, true>(a, st); break;
+            case 7: e2 = launch_score_v2<7, true>(a, st); break;
+            case 8: e2 = launch_score_v2<8, true>(a, st); break;
+            default: break;
+            }
+        }
+        if (e2 != cudaErrorNotSupported) return e2;
+    }
     const size_t psmem = (size_t)2 * a.d * sizeof(float);
     score_prologue_kernel<<<(unsigned)(a.G * a.nq), 256, psmem, st>>>(a.q, a.d, a.m, a.proj, a.proj_bf16, *a.tables,
                                                                       two, a.workspace);

@@ -293,6 +293,7 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
     a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
     if (!rq::make_rows64_tmap(&a.tmap_x, x, n / 64)) return RQ_ECUDA;
+    a.has_tmap_v = qjl && rq::make_vectors_tmap(&a.tmap_v, x, n / d, d);
     return cuda_status(rq::launch_quantize(a, stream));
 }
 

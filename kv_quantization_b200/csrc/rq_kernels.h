@@ -23,6 +23,8 @@ struct QuantArgs {
     uint16_t *qnorms;
     int num_sms;
     CUtensorMap tmap_x;        // input as [n/64][64] 16-bit rows, 256-row boxes, 128-byte swizzle
+    CUtensorMap tmap_v;        // input as {64, d/64, n/d} blocks, {64, 1, 128} boxes (tensor-core A layout)
+    bool has_tmap_v;
 };
 
 struct DequantArgs {

@@ -5,6 +5,7 @@
 #include "rq_qjl_mma.cuh"
 #include "rq_v2.cuh"
 #include "rq_qjl_v2.cuh"
+#include "rq_qjl_v3.cuh"
 
 namespace rq {
 
@@ -48,34 +49,35 @@ static cudaError_t launch_mma(const QuantTables &T, const void *x, int64_t nvec,
     return cudaGetLastError();
 }
 
-// Pipelined tensor-core paths for d = 128 (rq_qjl_v2.cuh); NotSupported when
-// the shape or the shared memory does not fit.
-template <int PW, bool BF16>
-static cudaError_t launch_qjl_v2(const QuantArgs &a, cudaStream_t st)
+// In-place pipelined fused quantize + sketch (rq_qjl_v3.cuh) for d = 128 / 256;
+// NotSupported when the shape or the shared memory does not fit.
+template <int D, int PW, bool BF16, int NS>
+static cudaError_t launch_qjl_v3_ns(const QuantArgs &a, size_t smem, cudaStream_t st)
 {
-    const QuantTables &T = *a.tables;
-    const int64_t tiles = (a.nblocks + 127) / 128;
-    const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
-    if (2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
-    size_t smem = qjl_v2_smem(0, PW, a.m, T, 3);
-    if (smem <= kMaxSmemPerBlock) {
-        auto kern = qjl_v2_quant_kernel<PW, BF16, 3>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_x, a.nblocks, T, static_cast<uint8_t *>(a.codes),
-                                                                a.norms, a.m, static_cast<const uint16_t *>(a.proj),
-                                                                a.qsigns, a.qnorms);
-        return cudaGetLastError();
-    }
-    smem = qjl_v2_smem(0, PW, a.m, T, 2);
-    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
-    auto kern = qjl_v2_quant_kernel<PW, BF16, 2>;
+    auto kern = qjl_v3_quant_kernel<D, PW, BF16, NS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_x, a.nblocks, T, static_cast<uint8_t *>(a.codes),
-                                                            a.norms, a.m, static_cast<const uint16_t *>(a.proj),
-                                                            a.qsigns, a.qnorms);
+    const int64_t tiles = (a.nblocks + 127) / 128;
+    const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_v, a.nblocks, *a.tables,
+                                                            static_cast<uint8_t *>(a.codes), a.norms, a.m,
+                                                            static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
     return cudaGetLastError();
+}
+
+template <int D, int PW, bool BF16>
+static cudaError_t launch_qjl_v3(const QuantArgs &a, cudaStream_t st)
+{
+    if constexpr (D != 128 && D != 256) {
+        return cudaErrorNotSupported;
+    } else {
+        if (!a.has_tmap_v || 2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
+        size_t smem = qjl_v3_smem(D, PW, a.m, *a.tables, 3);
+        if (smem <= kMaxSmemPerBlock) return launch_qjl_v3_ns<D, PW, BF16, 3>(a, smem, st);
+        smem = qjl_v3_smem(D, PW, a.m, *a.tables, 1);
+        if (smem <= kMaxSmemPerBlock) return launch_qjl_v3_ns<D, PW, BF16, 1>(a, smem, st);
+        return cudaErrorNotSupported;
+    }
 }
 
 template <bool BF16>
@@ -165,8 +167,8 @@ cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_
 #define RQ_CASE(PW)                                                                                       \
     case PW:                                                                                              \
         if (qjl) {                                                                                        \
-            if (RQ_D == 128) {                                                                            \
-                cudaError_t e2 = launch_qjl_v2<PW, RQ_BF16>(a, st);                                       \
+            {                                                                                             \
+                cudaError_t e2 = launch_qjl_v3<RQ_D, PW, RQ_BF16>(a, st);                                 \
                 if (e2 != cudaErrorNotSupported) return e2;                                               \
             }                                                                                             \
             cudaError_t e = launch_mma<RQ_D, PW, RQ_BF16, 0>(*a.tables, a.x, a.nblocks, a.codes, a.norms, a.m, \

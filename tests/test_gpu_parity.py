@@ -309,3 +309,33 @@ def test_score_two_stage(d):
     err = np.abs(scores.cpu().numpy().astype(np.float64) - want)
     tol = _score_tol(q16, G, nq, d, qn.cpu().numpy().view(np.uint16), norms.cpu().numpy().view(np.uint16))
     assert np.all(err <= tol), float((err / tol).max())
+
+
+@pytest.mark.parametrize("d,bits,m,nq,layout", [(128, 4, 128, 40, L.RQ_CODES_INT8), (64, 3, 72, 7, L.RQ_CODES_PACKED),
+                                                 (128, 5, 256, 33, L.RQ_CODES_PACKED)])
+def test_score_two_stage_shapes(d, bits, m, nq, layout):
+    """Query counts that are not multiples of 32, m not a multiple of 64,
+    int8 codes, and a ragged token tail."""
+    G, T = 3, 131
+    k = synth.normal((G, T, d), seed=16, device=DEV).reshape(-1)
+    q = synth.normal((G, nq, d), seed=17, device=DEV)
+    cent = L.rq_lloyd_max(bits)
+    S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
+    L.qjl_make_projection(8, m, d, S)
+    codes = torch.empty(L.rq_code_bytes(k.numel(), d, bits, layout), dtype=torch.uint8, device=DEV)
+    norms = torch.empty(G * T, dtype=torch.int16, device=DEV)
+    qs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=DEV)
+    qn = torch.empty(G * T, dtype=torch.int16, device=DEV)
+    L.rq_quantize_qjl(k, d, bits, layout, 1, 9, cent, m, S, codes, norms, qs, qn)
+    scores = torch.empty(G, nq, T, dtype=torch.float32, device=DEV)
+    ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4 + 1, dtype=torch.float32, device=DEV)
+    L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits, layout=layout,
+                use_signs=1, sign_seed=9, centroids=cent)
+    torch.cuda.synchronize()
+    q16 = u16(q)
+    want = O.score(q16, G, nq, d, m, u16(S), O.BF16, qs.cpu().numpy(), qn.cpu().numpy().view(np.uint16), T,
+                   codes=codes.cpu().numpy(), norms=norms.cpu().numpy().view(np.uint16), bits=bits,
+                   layout=layout, signs_diag=O.sign_diagonal(9, d), c32=cent)
+    err = np.abs(scores.cpu().numpy().astype(np.float64) - want)
+    tol = _score_tol(q16, G, nq, d, qn.cpu().numpy().view(np.uint16), norms.cpu().numpy().view(np.uint16))
+    assert np.all(err <= tol), float((err / tol).max())

@@ -124,7 +124,7 @@ def test_qjl_rejects_bad_m():
 
 
 def test_score_workspace_size_and_check():
-    assert L.qjl_score_workspace_bytes(8, 32, 256, 256) == 8 * 32 * 512 * 4
+    assert L.qjl_score_workspace_bytes(8, 32, 256, 256) >= 8 * 32 * 512 * 4
     small = FakeTensor(0x90000, numel=16)
     with pytest.raises(L.RQError) as e:
         L.qjl_score(FakeTensor(0x40000), 8, 32, 256, 256, FakeTensor(0x50000), FakeTensor(0x60000),
