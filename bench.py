@@ -130,6 +130,27 @@ def make_inputs(dev):
     return synth.student_t_outliers(ROWS, COLS, seed=1, device=dev).reshape(-1)
 
 
+def reduce_max_ms(total_ms, world, device=None):
+    """Max over ranks of the per-rank timed milliseconds (the job ends with its
+    slowest replica); identity on one rank."""
+    if world <= 1:
+        return float(total_ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank_step, world, steps, max_ms):
+    """Whole-job throughput: the units every replica processed / the max time."""
+    return units_per_rank_step * world * steps / (max_ms * 1e-3)
+
+
+def alg_bytes_quant(n, bits):
+    return n * 2 + n * bits / 8 + 2 * n / D
+
+
 def alg_bytes_quant_qjl(n, bits):
     return n * 2 + n * bits / 8 + 2 * n / D + n * M / (8 * D) + 2 * n / D
 
@@ -211,22 +232,17 @@ def run_device(args, rank, world):
         for k in range(n_ev):
             kern_ms[s][k] = evs[k][0].elapsed_time(evs[k][1])
         step_ms.append(sum(kern_ms[s]))
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-
+    total_ms = reduce_max_ms(sum(step_ms), world, dev)
     in_bytes = n * 2 * len(BITS)
-    value = in_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
+    value = job_rate(in_bytes, world, args.steps, total_ms) / 1e9
     hbm, tf, src = peaks()
     # dominant kernel: the larger of quantize_qjl / dequantize by total time
     q_ms = [statistics.mean(kern_ms[s][2 * i] for s in range(args.steps)) for i in range(len(BITS))]
     dq_ms = [statistics.mean(kern_ms[s][2 * i + 1] for s in range(args.steps)) for i in range(len(BITS))]
     if sum(q_ms) >= sum(dq_ms):
-        dom, alg, ms = "quantize_kernel<128,b,bf16,qjl>", sum(alg_bytes_quant_qjl(n, b) for b in BITS), sum(q_ms)
+        dom, alg, ms = "qjl_v3_quant_kernel<128,b,bf16,3>", sum(alg_bytes_quant_qjl(n, b) for b in BITS), sum(q_ms)
     else:
-        dom, alg, ms = "dequantize_kernel<128,b,bf16>", sum(alg_bytes_dequant(n, b) for b in BITS), sum(dq_ms)
+        dom, alg, ms = "dequantize_v2_kernel<128,b,bf16>", sum(alg_bytes_dequant(n, b) for b in BITS), sum(dq_ms)
     achieved = alg / (ms * 1e-3) / 1e9
     per_kernel = {f"quantize_qjl_b{b}_ms": round(q, 4) for b, q in zip(BITS, q_ms)}
     per_kernel.update({f"dequantize_b{b}_ms": round(q, 4) for b, q in zip(BITS, dq_ms)})
@@ -234,6 +250,33 @@ def run_device(args, rank, world):
                        for b, q in zip(BITS, q_ms)})
     per_kernel.update({f"dequantize_b{b}_gbs": round(alg_bytes_dequant(n, b) / (q * 1e-3) / 1e9, 1)
                        for b, q in zip(BITS, dq_ms)})
+
+    # quantize + dequantize alone (no QJL stage), same workload and cold L2
+    qd = {}
+    for b in BITS:
+        B = bufs[b]
+        tq, tdq = [], []
+        for _ in range(max(5, min(args.steps, 50))):
+            l2_flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            rq.rq_quantize(x, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], B["codes"], B["norms"])
+            e1.record(stream)
+            l2_flush()
+            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e2.record(stream)
+            rq.rq_dequantize(B["codes"], B["norms"], n, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], B["out"])
+            e3.record(stream)
+            torch.cuda.synchronize()
+            tq.append(e0.elapsed_time(e1))
+            tdq.append(e2.elapsed_time(e3))
+        mq, mdq = statistics.mean(tq), statistics.mean(tdq)
+        qd[f"b{b}"] = {"quantize_ms": round(mq, 4), "dequantize_ms": round(mdq, 4),
+                       "quantize_gbs": round(alg_bytes_quant(n, b) / (mq * 1e-3) / 1e9, 1),
+                       "dequantize_gbs": round(alg_bytes_dequant(n, b) / (mdq * 1e-3) / 1e9, 1),
+                       "input_gbs": round(n * 2 / ((mq + mdq) * 1e-3) / 1e9, 1),
+                       "pct_hbm": round(100 * (alg_bytes_quant(n, b) + alg_bytes_dequant(n, b)) /
+                                        ((mq + mdq) * 1e-3) / 1e9 / peaks()[0], 1)}
 
     # end to end through the public API with host buffers
     e2e = e2e_measure(args, x, S, tabs, bufs, dev)
@@ -250,6 +293,7 @@ def run_device(args, rank, world):
                      "frac": round(achieved / hbm, 4), "peak_source": src, "traffic": None,
                      "alg_bytes_per_step": alg},
         "kernels": per_kernel,
+        "quantize_dequantize_only": qd,
         "e2e": e2e,
         "gpu_launches": n_ev * args.steps,
         "clocks": clk.summary(),
