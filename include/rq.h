@@ -156,6 +156,30 @@ rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void 
                     int use_signs, uint64_t sign_seed, const float *centroids,
                     float *scores, void *workspace, size_t workspace_bytes, rq_stream_t stream);
 
+/* qjl_score without a caller-provided workspace.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory -- a serving engine that reserved all of its HBM for the KV
+ * cache at start-up and forbids later allocations, or a host that reaches this
+ * library through a plain-C plugin interface that passes device pointers but
+ * no allocator.  It computes exactly what qjl_score computes (same arguments
+ * minus workspace / workspace_bytes) and allocates nothing: its scratch is an
+ * 8 MiB array inside the library's own device image, which every GPU that
+ * loads the library holds until the process exits.
+ *   - Returns RQ_ESIZE when qjl_score_workspace_bytes(G, n_q, d, m) exceeds
+ *     8 MiB (8388608 bytes), before touching the GPU.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and remembers it; make that first call before any
+ *     stream capture.  RQ_ECUDA if the lookup fails.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents (nothing in it needs to start at zero).  Calls whose
+ *     work overlaps on the GPU -- e.g. on two streams without ordering between
+ *     them -- race on it; order them on one stream or with events. */
+rq_status qjl_score_noalloc(const void *q, int64_t G, int n_q, int d, int m, const void *proj, rq_dtype proj_dtype,
+                            const uint8_t *signs, const uint16_t *sk_norms, int64_t T,
+                            const void *codes, const uint16_t *norms, int bits, rq_layout layout,
+                            int use_signs, uint64_t sign_seed, const float *centroids,
+                            float *scores, rq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,8 @@ def lib() -> C.CDLL:
                 "qjl_score_workspace_bytes": (sz, [i64, i32, i32, i32]),
                 "qjl_score": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32, u64,
                                     fp, vp, vp, sz, vp]),
+                "qjl_score_noalloc": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32,
+                                            u64, fp, vp, vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -64,7 +66,8 @@ def lib() -> C.CDLL:
 def exported_symbols():
     """Names this binding expects librq.so to export."""
     return ["rq_status_string", "rq_device_error", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
-            "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score"]
+            "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score",
+            "qjl_score_noalloc"]
 
 
 def status_string(status: int) -> str:
@@ -163,3 +166,16 @@ def qjl_score(q, G, n_q, d, m, proj, signs, sk_norms, T, scores, workspace, code
         _dev(q), G, n_q, d, m, _dev(proj), _dtype_code(proj), _dev(signs), _dev(sk_norms), T, _dev(codes),
         _dev(norms), bits, layout, int(use_signs), sign_seed, cp, _dev(scores), _dev(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def qjl_score_noalloc(q, G, n_q, d, m, proj, signs, sk_norms, T, scores, codes=None, norms=None, bits=0,
+                      layout=RQ_CODES_PACKED, use_signs=0, sign_seed=0, centroids=None, stream=None):
+    """qjl_score with the library's own fixed 8 MiB device scratch instead of a
+    caller workspace, for callers that cannot allocate device memory."""
+    if centroids is None:
+        cp = None
+    else:
+        c, cp = _table(centroids)
+    _check("qjl_score_noalloc", lib().qjl_score_noalloc(
+        _dev(q), G, n_q, d, m, _dev(proj), _dtype_code(proj), _dev(signs), _dev(sk_norms), T, _dev(codes),
+        _dev(norms), bits, layout, int(use_signs), sign_seed, cp, _dev(scores), _stream(stream)))
