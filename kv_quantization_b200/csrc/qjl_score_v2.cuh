@@ -76,6 +76,7 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
     float *pinv = pr + kSc2PrologueQ * d;
     const int64_t g = blockIdx.x;
     const int q0 = blockIdx.y * kSc2PrologueQ;
+    const int zs = blockIdx.z, nz = gridDim.z;        // slice of the S q outputs (z = 0 also rotates)
     const int nqc = min(kSc2PrologueQ, nq - q0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int idx = tid; idx < kSc2PrologueQ * d; idx += blockDim.x) {
@@ -93,10 +94,10 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
         if (lane == 0) {
             const float qn = sqrtf(sum);
             pinv[qi] = qn > 0.0f ? 1.0f / qn : 0.0f;
-            if (qi < nqc) wsN[(int64_t)g * nq + q0 + qi] = qn;
+            if (qi < nqc && zs == 0) wsN[(int64_t)g * nq + q0 + qi] = qn;
         }
     }
-    if (two) {
+    if (two && zs == 0) {
         for (int h = 1; h < d; h *= 2) {
             __syncthreads();
             for (int p = tid; p < kSc2PrologueQ * d / 2; p += blockDim.x) {
@@ -110,12 +111,14 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
     }
     __syncthreads();
     const int kb = sc2_kb(d, m, two), off = two ? d : 0;
-    if (two)
+    if (two && zs == 0)
         for (int idx = tid; idx < nqc * d; idx += blockDim.x) {
             const int qi = idx / d, j = idx % d;
             wsB[((int64_t)g * nq + q0 + qi) * kb + j] = __half_as_ushort(__float2half_rn(pr[idx] * pinv[qi]));
         }
-    for (int i = tid; i < sc2_m64(m); i += blockDim.x) {
+    const int per = (sc2_m64(m) + nz - 1) / nz;
+    const int i_lo = zs * per, i_hi = min(sc2_m64(m), i_lo + per);
+    for (int i = i_lo + tid; i < i_hi; i += blockDim.x) {
         float acc[kSc2PrologueQ];
 #pragma unroll
         for (int qi = 0; qi < kSc2PrologueQ; ++qi) acc[qi] = 0.0f;

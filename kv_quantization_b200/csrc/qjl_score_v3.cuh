@@ -61,7 +61,7 @@ __host__ __device__ inline size_t sc3_smem(int nq, int d, int m, bool two, int p
     b += (size_t)nq32 * kb * 2;                                    // B
     b += (size_t)256 * 8 * 16;                                     // sign LUT
     if (two) b += pw <= 4 ? ((size_t)1 << (2 * pw)) * 32 * 4 : ((size_t)1 << pw) * 32 * 2;
-    b += 2 * (size_t)128 * sc3_row_bytes(d, m, two, pw);           // records, 2 tiles
+    b += 3 * (size_t)128 * sc3_row_bytes(d, m, two, pw);           // records, 3 tiles
     return b + 8 * (2 * kSc3Ring + 5) + 16;
 }
 
@@ -87,7 +87,7 @@ score_v3_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
     uint32_t *clut = reinterpret_cast<uint32_t *>(slut + 256 * 8);
     const size_t clut_bytes = TWO ? (PW <= 4 ? ((size_t)1 << (2 * PW)) * 32 * 4 : ((size_t)1 << PW) * 32 * 2) : 0;
     uint8_t *srec = reinterpret_cast<uint8_t *>(clut) + clut_bytes;
-    uint64_t *a_full = reinterpret_cast<uint64_t *>(srec + 2 * 128 * rowb);
+    uint64_t *a_full = reinterpret_cast<uint64_t *>(srec + 3 * 128 * rowb);
     uint64_t *a_empty = a_full + kSc3Ring;
     uint64_t *acc_full = a_empty + kSc3Ring;
     uint64_t *acc_empty = acc_full + 2;
@@ -170,11 +170,13 @@ score_v3_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
         };
         if (it0 < it1) prefetch(it0, 0);
         cp_async_commit();
+        if (it0 + 1 < it1) prefetch(it0 + 1, 1);
+        cp_async_commit();
         int64_t chunk = 0;
         for (int64_t it = it0; it < it1 && ok; ++it) {
-            const int rb = (int)((it - it0) & 1);
-            cp_async_wait_all();                   // this tile's record is in shared memory
-            if (it + 1 < it1) prefetch(it + 1, rb ^ 1);
+            const int rb = (int)((it - it0) % 3);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");   // this tile's record is in shared memory
+            if (it + 2 < it1) prefetch(it + 2, (int)((it + 2 - it0) % 3));
             cp_async_commit();
             const int64_t t = (it % tiles_per_g) * 128 + r;
             const bool tv = t < T_len;
@@ -316,30 +318,45 @@ score_v3_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
         const int quarter = warp & 3;              // TMEM lanes this warp may read
         const int r = quarter * 32 + lane;         // token row
         const float kq = 1.2533141373155002512f / (float)m;
+        int64_t qn_g = -1;
+        float qn_reg[4] = {0.0f, 0.0f, 0.0f, 0.0f}; // lane i holds ||q|| of queries i, 32+i, 64+i, 96+i
         for (int64_t it = it0; it < it1 && ok; ++it) {
             const int64_t g = it / tiles_per_g, t = (it % tiles_per_g) * 128 + r;
             const int a = (int)((it - it0) & 1);
             const int64_t ause = (it - it0) >> 1;
+            const bool tin = t < T_len;
+            const int64_t kt = g * T_len + (tin ? t : 0);
+            // loads that do not depend on the accumulator go out before the wait
+            const uint16_t skn = tin ? __ldg(sk_norms + kt) : (uint16_t)0;
+            const uint16_t n1 = (TWO && tin) ? __ldg(norms + kt) : (uint16_t)0;
+            if (g != qn_g) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int qi = 32 * k + lane;
+                    qn_reg[k] = qi < nq ? __ldg(wsN + g * nq + qi) : 0.0f;
+                }
+                qn_g = g;
+            }
             if (ok && !mbar_wait(&acc_full[a], (uint32_t)(ause & 1))) ok = false;
             tc_fence_after();
-            const bool tv = ok && t < T_len;
-            const int64_t kt = g * T_len + (tv ? t : 0);
-            const float a2 = tv ? __fmul_rn(kq, h16_to_f32(__ldg(sk_norms + kt))) : 0.0f;
-            const float a1 = (TWO && tv) ? __fmul_rn(h16_to_f32(__ldg(norms + kt)), 1.0f / (float)d) : 0.0f;
+            const bool tv = ok && tin;
+            const float a2 = __fmul_rn(kq, h16_to_f32(skn));
+            const float a1 = TWO ? __fmul_rn(h16_to_f32(n1), 1.0f / (float)d) : 0.0f;
             const uint32_t col1 = (uint32_t)(a * 2 * nq32), col2 = col1 + (uint32_t)nq32;
             for (int q0 = 0; q0 < nq32; q0 += 32) {
                 uint32_t r1[32], r2[32];
                 tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + col2 + (uint32_t)q0, r2);
                 if (TWO) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + col1 + (uint32_t)q0, r1);
                 tmem_ld_wait();
-                const float *qn = wsN + g * nq + q0;
+                const float qn_mine = qn_reg[q0 >> 5];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int qi = q0 + i;
+                    const float qn = __shfl_sync(0xffffffffu, qn_mine, i);
                     if (tv && qi < nq) {
-                        float s = __fmul_rn(a2, __uint_as_float(r2[i]));
-                        if (TWO) s = __fmaf_rn(a1, __uint_as_float(r1[i]), s);
-                        scores[((int64_t)g * nq + qi) * T_len + t] = __fmul_rn(s, __ldg(qn + i));
+                        float sv = __fmul_rn(a2, __uint_as_float(r2[i]));
+                        if (TWO) sv = __fmaf_rn(a1, __uint_as_float(r1[i]), sv);
+                        scores[((int64_t)g * nq + qi) * T_len + t] = __fmul_rn(sv, qn);
                     }
                 }
             }

@@ -208,6 +208,19 @@ bool rq::make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool rq::make_proj_tmap(CUtensorMap *map, const void *ptr, int m, int d, int box_rows)
+{
+    auto enc = tmap_encoder();
+    if (!enc || m <= 0 || d % 64 || box_rows <= 0 || box_rows > 256) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)m};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 extern "C" {
 
 const char *rq_status_string(int status)
@@ -363,6 +376,10 @@ rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m,
     a.norms = norms; a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
     a.has_tmap_k = rq::make_vectors_tmap(&a.tmap_k, x, n_vec, d);
+    {
+        const int m16 = (m + 15) & ~15;
+        a.has_tmap_s = (m16 <= 256 || m16 % 256 == 0) && rq::make_proj_tmap(&a.tmap_s, proj, m, d, m16 < 256 ? m16 : 256);
+    }
     return cuda_status(rq::launch_sketch(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -50,6 +50,8 @@ struct SketchArgs {
     int num_sms;
     CUtensorMap tmap_k;        // keys as {64, d/64, n_vec} 16-bit, {64, 1, 128} boxes, 128-byte swizzle
     bool has_tmap_k;
+    CUtensorMap tmap_s;        // S as [m][d] 16-bit, {64, rows} boxes, 128-byte swizzle (B layout)
+    bool has_tmap_s;
 };
 
 struct ScoreArgs {
@@ -83,6 +85,8 @@ bool make_rows64_tmap(CUtensorMap *map, const void *ptr, int64_t rows);
 // Encode vectors[n][d] (16-bit) as {64, d/64, n} with {64, 1, 128} boxes:
 // one box is one 64-column region of 128 vectors, the tensor-core A layout.
 bool make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d);
+// Encode S[m][d] (16-bit) with {64 columns, box_rows rows} boxes (B operand layout).
+bool make_proj_tmap(CUtensorMap *map, const void *ptr, int m, int d, int box_rows);
 size_t dequantize_smem_bytes(int d);
 
 }  // namespace rq

@@ -45,6 +45,26 @@ __host__ __device__ inline size_t qjl_v2_smem(int mode, int pw, int m, const Qua
     return b + 8 * (stages + 2) + 16;
 }
 
+// Bit i of the result = (v[i] >= 0) for 32 fp32 values.  Adding +0 maps -0
+// to +0 (and leaves every other value unchanged), so the bit is the inverted
+// sign bit; the 32 shifts are independent and combine in an OR tree.
+__device__ __forceinline__ uint32_t sign_word(const uint32_t *v)
+{
+    uint32_t part[8];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        uint32_t b[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = 4 * g + k;
+            const uint32_t x = __float_as_uint(__fadd_rn(__uint_as_float(v[i]), 0.0f));
+            b[k] = (x >> 31) << i;                       // 1 where negative
+        }
+        part[g] = (b[0] | b[1]) | (b[2] | b[3]);
+    }
+    return ~(((part[0] | part[1]) | (part[2] | part[3])) | ((part[4] | part[5]) | (part[6] | part[7])));
+}
+
 // Sign-pack epilogue of one 128-vector tile from TMEM accumulator columns
 // [col0, col0 + m16).
 __device__ __forceinline__ void qjl_v2_epilogue(uint32_t tmem, uint32_t col0, int m, int m16, int64_t tok0,
@@ -58,9 +78,7 @@ __device__ __forceinline__ void qjl_v2_epilogue(uint32_t tmem, uint32_t col0, in
         uint32_t acc[32];
         tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + col0 + (uint32_t)c0, acc);
         tmem_ld_wait();
-        uint32_t word = 0u;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) word |= (__uint_as_float(acc[i]) >= 0.0f ? 1u : 0u) << i;
+        const uint32_t word = sign_word(acc);
         if (tv && c0 < m) {
             const int nb = min(4, (m - c0) / 8);
             if (nb == 4 && (m & 31) == 0) {

@@ -6,6 +6,7 @@
 #include "rq_v2.cuh"
 #include "rq_qjl_v2.cuh"
 #include "rq_qjl_v3.cuh"
+#include "rq_sketch_v3.cuh"
 
 namespace rq {
 
@@ -72,7 +73,9 @@ static cudaError_t launch_qjl_v3(const QuantArgs &a, cudaStream_t st)
         return cudaErrorNotSupported;
     } else {
         if (!a.has_tmap_v || 2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
-        size_t smem = qjl_v3_smem(D, PW, a.m, *a.tables, 3);
+        size_t smem = qjl_v3_smem(D, PW, a.m, *a.tables, 5);
+        if (smem <= kMaxSmemPerBlock) return launch_qjl_v3_ns<D, PW, BF16, 5>(a, smem, st);
+        smem = qjl_v3_smem(D, PW, a.m, *a.tables, 3);
         if (smem <= kMaxSmemPerBlock) return launch_qjl_v3_ns<D, PW, BF16, 3>(a, smem, st);
         smem = qjl_v3_smem(D, PW, a.m, *a.tables, 1);
         if (smem <= kMaxSmemPerBlock) return launch_qjl_v3_ns<D, PW, BF16, 1>(a, smem, st);
@@ -81,13 +84,37 @@ static cudaError_t launch_qjl_v3(const QuantArgs &a, cudaStream_t st)
 }
 
 template <bool BF16>
+static cudaError_t launch_sketch_v3(const SketchArgs &a, cudaStream_t st)
+{
+    if (!a.has_tmap_k || !a.has_tmap_s || 2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
+    const int64_t tiles = (a.nvec + 127) / 128;
+    const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
+    size_t smem = sketch_v3_smem(a.m, 5);
+    auto kern = sketch_v3_kernel<BF16, 5>;
+    if (smem > kMaxSmemPerBlock) {
+        smem = sketch_v3_smem(a.m, 3);
+        kern = sketch_v3_kernel<BF16, 3>;
+    }
+    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kSk3Warps * 32, smem, st>>>(a.tmap_k, a.tmap_s, a.nvec, a.m, a.signs,
+                                                                        a.norms);
+    return cudaGetLastError();
+}
+
+template <bool BF16>
 static cudaError_t launch_sketch_v2(const SketchArgs &a, cudaStream_t st)
 {
     if (!a.has_tmap_k || 2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
     QuantTables T{};
-    const size_t smem = qjl_v2_smem(1, 1, a.m, T, 3);
+    size_t smem = qjl_v2_smem(1, 1, a.m, T, 5);
+    auto kern = qjl_v2_sketch_kernel<BF16, 5>;
+    if (smem > kMaxSmemPerBlock) {
+        smem = qjl_v2_smem(1, 1, a.m, T, 3);
+        kern = qjl_v2_sketch_kernel<BF16, 3>;
+    }
     if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
-    auto kern = qjl_v2_sketch_kernel<BF16, 3>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (a.nvec + 127) / 128;
@@ -198,6 +225,8 @@ cudaError_t RQ_CAT(launch_dequantize, RQ_D, RQ_DT)(const DequantArgs &a, cudaStr
 cudaError_t RQ_CAT(launch_sketch, RQ_D, RQ_DT)(const SketchArgs &a, cudaStream_t st)
 {
     if (RQ_D == 128) {
+        cudaError_t e3 = launch_sketch_v3<RQ_BF16>(a, st);
+        if (e3 != cudaErrorNotSupported) return e3;
         cudaError_t e2 = launch_sketch_v2<RQ_BF16>(a, st);
         if (e2 != cudaErrorNotSupported) return e2;
     }
