@@ -240,9 +240,9 @@ def run_device(args, rank, world):
     q_ms = [statistics.mean(kern_ms[s][2 * i] for s in range(args.steps)) for i in range(len(BITS))]
     dq_ms = [statistics.mean(kern_ms[s][2 * i + 1] for s in range(args.steps)) for i in range(len(BITS))]
     if sum(q_ms) >= sum(dq_ms):
-        dom, alg, ms = "qjl_v3_quant_kernel<128,b,bf16,3>", sum(alg_bytes_quant_qjl(n, b) for b in BITS), sum(q_ms)
+        dom, alg, ms = "qjl_v6_quant_kernel<b,bf16,signs> (d=128)", sum(alg_bytes_quant_qjl(n, b) for b in BITS), sum(q_ms)
     else:
-        dom, alg, ms = "dequantize_v2_kernel<128,b,bf16>", sum(alg_bytes_dequant(n, b) for b in BITS), sum(dq_ms)
+        dom, alg, ms = "dequantize_v5_kernel<b,bf16,signs> (d=128)", sum(alg_bytes_dequant(n, b) for b in BITS), sum(dq_ms)
     achieved = alg / (ms * 1e-3) / 1e9
     per_kernel = {f"quantize_qjl_b{b}_ms": round(q, 4) for b, q in zip(BITS, q_ms)}
     per_kernel.update({f"dequantize_b{b}_ms": round(q, 4) for b, q in zip(BITS, dq_ms)})

@@ -22,9 +22,11 @@
  * Conventions shared by every entry point
  *   - Pointers named x, codes, norms, out, proj, signs, scores, q and workspace
  *     are DEVICE pointers owned by the caller; `centroids` is a HOST pointer.
- *     The library keeps no pointer after a call returns, allocates no device
- *     memory and keeps no global state besides one device error word
- *     (rq_device_error).
+ *     The library keeps no pointer after a call returns and allocates no
+ *     device memory.  Its only global state: one device error word
+ *     (rq_device_error), the fixed scratch array of qjl_score_noalloc, and a
+ *     mutex-guarded host cache of the last few per-call lookup tables (a pure
+ *     function of centroids, bits, d and the sign seed).
  *   - Every call validates its arguments on the host, then enqueues its
  *     kernels asynchronously on `stream` (0 = legacy default stream) and
  *     returns.  Kernel faults surface at the caller's next synchronisation.
@@ -106,7 +108,9 @@ rq_status rq_quantize(const void *x, rq_dtype dtype, int64_t n, int d, int bits,
                       void *codes, uint16_t *norms, rq_stream_t stream);
 
 /* Reconstruct n values into out (out_dtype) from codes and fp16 norms written
- * by rq_quantize with the same d, bits, layout, signs and centroids. */
+ * by rq_quantize with the same d, bits, layout, signs and centroids.  An
+ * int8-layout byte >= 2^bits is not a code rq_quantize writes: the values of
+ * its block are then unspecified, but no memory outside the arguments is read. */
 rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int d, int bits,
                         rq_layout layout, int use_signs, uint64_t sign_seed, const float *centroids,
                         void *out, rq_dtype out_dtype, rq_stream_t stream);

@@ -12,6 +12,7 @@ from __future__ import annotations
 import concurrent.futures as cf
 import glob
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -51,6 +52,27 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
+_INCLUDE_RE = re.compile(r'^\s*#\s*include\s+"([^"]+)"', re.M)
+
+
+def _closure(src):
+    """The source and every local header it includes, transitively."""
+    seen, todo = set(), [src]
+    while todo:
+        f = todo.pop()
+        if f in seen or not os.path.exists(f):
+            continue
+        seen.add(f)
+        with open(f, encoding="utf-8", errors="replace") as fh:
+            for name in _INCLUDE_RE.findall(fh.read()):
+                for d in (os.path.dirname(f), CSRC, INCLUDE):
+                    cand = os.path.join(d, name)
+                    if os.path.exists(cand):
+                        todo.append(os.path.normpath(cand))
+                        break
+    return seen
+
+
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     if not force and up_to_date():
         return LIB
@@ -59,6 +81,9 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     def compile_one(src):
         obj = os.path.join(OBJ, os.path.basename(src) + ".o")
+        if not force and not extra_flags and os.path.exists(obj) and \
+                all(os.path.getmtime(p) <= os.path.getmtime(obj) for p in _closure(src)):
+            return obj                              # nothing it depends on changed
         cmd = [cc, *ARCH, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:

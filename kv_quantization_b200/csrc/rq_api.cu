@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <limits>
+#include <mutex>
 #include <vector>
 
 #include <cuda.h>
@@ -125,6 +126,77 @@ bool build_lut(const float *t, int nb, QuantTables &T)
     return false;
 }
 
+// The device's saturating-grid cell function: fma.rn.sat (clamp to [0, 1],
+// NaN to 0) then an fma that rounds fs * k to an integer in the low mantissa
+// bits of kLutMagic.
+int sat_cell(float y, float a, float b, float k)
+{
+    float f = std::fmaf(y, a, b);
+    f = f > 0.0f ? (f < 1.0f ? f : 1.0f) : 0.0f;
+    const float g = std::fmaf(f, k, rq::kLutMagic);
+    uint32_t gb, mb;
+    const float magic = rq::kLutMagic;
+    std::memcpy(&gb, &g, 4);
+    std::memcpy(&mb, &magic, 4);
+    return (int)(gb - mb);
+}
+
+// Saturating-grid LUT over [t_0 - w, t_last + w] with cell width w below the
+// smallest boundary gap; every cell's y-interval is found by bisection on the
+// float line and checked to hold at most one boundary.
+bool build_sat_lut(const float *t, int nb, QuantTables &T)
+{
+    if (nb < 1) return false;
+    double min_gap = INFINITY;
+    for (int k = 0; k + 1 < nb; ++k) min_gap = std::fmin(min_gap, (double)t[k + 1] - (double)t[k]);
+    if (!(min_gap > 0)) return false;
+    if (!std::isfinite(min_gap)) min_gap = 1.0;
+    const float lo_lim = -1.0e5f, hi_lim = 1.0e5f;
+    for (int attempt = 0; attempt < 64; ++attempt) {
+        const double w = min_gap / (1.25 + 0.125 * attempt);
+        const double ylo = (double)t[0] - w, yhi = (double)t[nb - 1] + w;
+        const int kcells = (int)std::ceil((yhi - ylo) / w);
+        if (kcells + 1 > rq::kMaxLutCells) return false;
+        const float a = (float)(1.0 / (yhi - ylo));
+        const float b = (float)(-ylo / (yhi - ylo));
+        const float k = (float)kcells;
+        const int cells = kcells + 1;
+        if (!(a > 0) || !std::isfinite(a) || !std::isfinite(b)) return false;
+        std::vector<float> lo(cells + 1);
+        lo[0] = -INFINITY;
+        lo[cells] = INFINITY;
+        for (int j = 1; j < cells; ++j) {
+            int64_t l = fkey(lo_lim), h = fkey(hi_lim);
+            if (sat_cell(keyf(h), a, b, k) < j) { lo[j] = INFINITY; continue; }
+            while (l < h) {
+                const int64_t mid = l + (h - l) / 2;
+                if (sat_cell(keyf(mid), a, b, k) >= j) h = mid; else l = mid + 1;
+            }
+            lo[j] = keyf(l);
+        }
+        bool ok = sat_cell(keyf(fkey(lo_lim)), a, b, k) == 0 && sat_cell(keyf(fkey(hi_lim)), a, b, k) == cells - 1;
+        for (int j = 0; j < cells && ok; ++j) {
+            int below = 0, inside = 0;
+            float cand = INFINITY;
+            for (int q = 0; q < nb; ++q) {
+                if (t[q] < lo[j]) ++below;
+                else if (t[q] < lo[j + 1]) { ++inside; cand = t[q]; }
+            }
+            if (inside > 1) ok = false;
+            T.sat_base[j] = (uint32_t)below;
+            T.sat_t[j] = inside ? cand : INFINITY;
+        }
+        if (ok) {
+            T.sat_a = a;
+            T.sat_b = b;
+            T.sat_k = k;
+            T.sat_cells = cells;
+            return true;
+        }
+    }
+    return false;
+}
+
 // Validate a host centroid table and fill the per-call tables.
 rq_status make_tables(const float *centroids, int bits, int d, int use_signs, uint64_t sign_seed,
                       QuantTables &T)
@@ -144,6 +216,7 @@ rq_status make_tables(const float *centroids, int bits, int d, int use_signs, ui
     }
     T.bound[K - 1] = INFINITY;
     if (!build_lut(T.bound, K - 1, T)) T.lut_cells = 0;
+    if (!build_sat_lut(T.bound, K - 1, T)) T.sat_cells = 0;
     if (use_signs) {
         for (int w = 0; w < d / 64; ++w) {
             const uint64_t r = splitmix64(sign_seed, (uint64_t)w);
@@ -151,6 +224,51 @@ rq_status make_tables(const float *centroids, int bits, int d, int use_signs, ui
             T.sign_words[2 * w + 1] = (uint32_t)(r >> 32);
         }
     }
+    return RQ_OK;
+}
+
+// The tables depend only on (centroids, bits, d, signs, seed) and take tens of
+// microseconds of host time to build (the LUT grids are verified by bisection
+// on the float line), so the last few are kept: a caller that quantizes
+// layer after layer with one configuration pays for them once.
+struct TableCacheEntry {
+    bool valid;
+    int bits, d, use_signs;
+    uint64_t seed;
+    float centroids[rq::kMaxLevels];
+    QuantTables T;
+};
+constexpr int kTableCache = 8;
+std::mutex g_table_mutex;
+TableCacheEntry g_table_cache[kTableCache];
+int g_table_next = 0;
+
+rq_status tables_for(const float *centroids, int bits, int d, int use_signs, uint64_t sign_seed, QuantTables &T)
+{
+    if (!centroids || bits < 1 || bits > 8) return RQ_EINVAL;
+    const int K = 1 << bits;
+    const uint64_t seed = use_signs ? sign_seed : 0;
+    {
+        std::lock_guard<std::mutex> lock(g_table_mutex);
+        for (const TableCacheEntry &e : g_table_cache)
+            if (e.valid && e.bits == bits && e.d == d && e.use_signs == (use_signs != 0) && e.seed == seed &&
+                std::memcmp(e.centroids, centroids, sizeof(float) * K) == 0) {
+                T = e.T;
+                return RQ_OK;
+            }
+    }
+    const rq_status s = make_tables(centroids, bits, d, use_signs, sign_seed, T);
+    if (s) return s;
+    std::lock_guard<std::mutex> lock(g_table_mutex);
+    TableCacheEntry &e = g_table_cache[g_table_next];
+    g_table_next = (g_table_next + 1) % kTableCache;
+    e.valid = true;
+    e.bits = bits;
+    e.d = d;
+    e.use_signs = use_signs != 0;
+    e.seed = seed;
+    std::memcpy(e.centroids, centroids, sizeof(float) * K);
+    e.T = T;
     return RQ_OK;
 }
 
@@ -195,13 +313,13 @@ bool rq::make_rows64_tmap(CUtensorMap *map, const void *ptr, int64_t rows)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool rq::make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d)
+bool rq::make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d, int box_rows)
 {
     auto enc = tmap_encoder();
-    if (!enc || n <= 0 || n >= ((int64_t)1 << 31) || d % 64) return false;
+    if (!enc || n <= 0 || n >= ((int64_t)1 << 31) || d % 64 || box_rows <= 0 || box_rows > 256) return false;
     const cuuint64_t dims[3] = {64, (cuuint64_t)(d / 64), (cuuint64_t)n};
     const cuuint64_t strides[2] = {128, (cuuint64_t)d * 2};
-    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -297,7 +415,7 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
     if (!aligned16(x) || !aligned16(codes) || !aligned16(norms)) return RQ_EALIGN;
     if (qjl && (!aligned16(proj) || !aligned16(qjl_signs) || !aligned16(qjl_norms))) return RQ_EALIGN;
     QuantTables T;
-    s = make_tables(centroids, bits, d, use_signs, sign_seed, T);
+    s = tables_for(centroids, bits, d, use_signs, sign_seed, T);
     if (s) return s;
     rq::QuantArgs a{};
     a.x = x; a.nblocks = n / d; a.d = d; a.pw = layout == RQ_CODES_INT8 ? 8 : bits; a.bf16 = dtype == RQ_BF16;
@@ -307,6 +425,7 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
     if (a.num_sms <= 0) return RQ_ECUDA;
     if (!rq::make_rows64_tmap(&a.tmap_x, x, n / 64)) return RQ_ECUDA;
     a.has_tmap_v = qjl && rq::make_vectors_tmap(&a.tmap_v, x, n / d, d);
+    a.has_tmap_v32 = !qjl && d == 128 && rq::make_vectors_tmap(&a.tmap_v32, x, n / d, d, 32);
     return cuda_status(rq::launch_quantize(a, stream));
 }
 
@@ -339,7 +458,7 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
     if (!codes || !norms || !out) return RQ_EINVAL;
     if (!aligned16(codes) || !aligned16(norms) || !aligned16(out)) return RQ_EALIGN;
     QuantTables T;
-    s = make_tables(centroids, bits, d, use_signs, sign_seed, T);
+    s = tables_for(centroids, bits, d, use_signs, sign_seed, T);
     if (s) return s;
     rq::DequantArgs a{};
     a.codes = codes; a.norms = norms; a.nblocks = n / d; a.d = d; a.pw = layout == RQ_CODES_INT8 ? 8 : bits;
@@ -347,6 +466,7 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
     a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
     if (!rq::make_rows64_tmap(&a.tmap_out, out, n / 64)) return RQ_ECUDA;
+    a.has_tmap_out32 = d == 128 && rq::make_vectors_tmap(&a.tmap_out32, out, n / d, d, 32);
     return cuda_status(rq::launch_dequantize(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -425,7 +545,7 @@ rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void 
         if (s) return s;
         if (!norms) return RQ_EINVAL;
         if (!aligned16(codes) || !aligned16(norms)) return RQ_EALIGN;
-        s = make_tables(centroids, bits, d, use_signs, sign_seed, T);
+        s = tables_for(centroids, bits, d, use_signs, sign_seed, T);
         if (s) return s;
         pw = layout == RQ_CODES_INT8 ? 8 : bits;
     }

@@ -25,6 +25,8 @@ struct QuantArgs {
     CUtensorMap tmap_x;        // input as [n/64][64] 16-bit rows, 256-row boxes, 128-byte swizzle
     CUtensorMap tmap_v;        // input as {64, d/64, n/d} blocks, {64, 1, 128} boxes (tensor-core A layout)
     bool has_tmap_v;
+    CUtensorMap tmap_v32;      // the same view with {64, 1, 32} boxes (one warp's 32-block chunk)
+    bool has_tmap_v32;
 };
 
 struct DequantArgs {
@@ -37,6 +39,8 @@ struct DequantArgs {
     void *out;
     int num_sms;
     CUtensorMap tmap_out;      // output as [n/64][64] 16-bit rows, 256-row boxes, 128-byte swizzle
+    CUtensorMap tmap_out32;    // output as {64, d/64, n/d} blocks, {64, 1, 32} boxes
+    bool has_tmap_out32;
 };
 
 struct SketchArgs {
@@ -82,9 +86,10 @@ size_t quantize_smem_bytes(int d, bool qjl);
 // Encode the [rows][64] 16-bit row view of `ptr` as a TMA map (256-row boxes,
 // 128-byte swizzle); false if the driver refuses it.
 bool make_rows64_tmap(CUtensorMap *map, const void *ptr, int64_t rows);
-// Encode vectors[n][d] (16-bit) as {64, d/64, n} with {64, 1, 128} boxes:
-// one box is one 64-column region of 128 vectors, the tensor-core A layout.
-bool make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d);
+// Encode vectors[n][d] (16-bit) as {64, d/64, n} with {64, 1, box_rows} boxes:
+// one box is one 64-column region of box_rows vectors (box_rows = 128: the
+// tensor-core A layout).
+bool make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d, int box_rows = 128);
 // Encode S[m][d] (16-bit) with {64 columns, box_rows rows} boxes (B operand layout).
 bool make_proj_tmap(CUtensorMap *map, const void *ptr, int m, int d, int box_rows);
 size_t dequantize_smem_bytes(int d);

@@ -23,6 +23,15 @@ struct QuantTables {
     float lut_b;
     int lut_cells;                   // 0: use the binary search over bound[]
     int levels;                      // K = 2^bits
+    // Saturating-grid LUT (one-block-per-thread kernels):
+    //   cell = bits(fma(sat(fma(y, sat_a, sat_b)), sat_k, magic)) - bits(magic), in [0, sat_cells)
+    // where sat() clamps to [0, 1]; no cell holds more than one boundary.
+    float sat_t[kMaxLutCells];       // per cell: the one boundary inside it, or +inf
+    uint32_t sat_base[kMaxLutCells]; // per cell: #boundaries below the cell
+    float sat_a;
+    float sat_b;
+    float sat_k;                     // sat_cells - 1
+    int sat_cells;                   // 0: no such grid (the caller takes another kernel)
 };
 
 }  // namespace rq

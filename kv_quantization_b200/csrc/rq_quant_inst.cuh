@@ -6,6 +6,8 @@
 #include "rq_v2.cuh"
 #include "rq_qjl_v2.cuh"
 #include "rq_qjl_v3.cuh"
+#include "rq_v5.cuh"
+#include "rq_v6.cuh"
 #include "rq_sketch_v3.cuh"
 
 namespace rq {
@@ -180,6 +182,81 @@ static cudaError_t launch_sk(const SketchArgs &a, cudaStream_t st)
     return cudaGetLastError();
 }
 
+// d = 128 kernels of rq_v5.cuh / rq_v6.cuh; NotSupported when the saturating
+// grid or the shared memory does not fit (the caller then takes the older
+// general-d kernels).
+
+template <int D, int PW, bool BF16>
+static cudaError_t launch_q5(const QuantArgs &a, cudaStream_t st)
+{
+    if constexpr (D != 128) {
+        return cudaErrorNotSupported;
+    } else {
+        if (!a.has_tmap_v32 || a.tables->sat_cells <= 0) return cudaErrorNotSupported;
+        const size_t smem = quantize_v5_smem(*a.tables);
+        if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+        const bool signs = a.tables->sign_words[0] | a.tables->sign_words[1] | a.tables->sign_words[2] |
+                           a.tables->sign_words[3];
+        auto kern = signs ? quantize_v5_kernel<PW, BF16, true> : quantize_v5_kernel<PW, BF16, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t chunks = (a.nblocks + 31) / 32;
+        const int64_t want = (chunks + kW5 - 1) / kW5;
+        const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
+        kern<<<(unsigned)(grid > 0 ? grid : 1), kW5 * 32, smem, st>>>(a.tmap_v32, a.nblocks, *a.tables,
+                                                                     static_cast<uint8_t *>(a.codes), a.norms);
+        return cudaGetLastError();
+    }
+}
+
+template <int D, int PW, bool BF16>
+static cudaError_t launch_dq5(const DequantArgs &a, cudaStream_t st)
+{
+    if constexpr (D != 128) {
+        return cudaErrorNotSupported;
+    } else {
+        if (!a.has_tmap_out32) return cudaErrorNotSupported;
+        const size_t smem = dequantize_v5_smem(PW, a.tables->levels);
+        if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+        const bool signs = a.tables->sign_words[0] | a.tables->sign_words[1] | a.tables->sign_words[2] |
+                           a.tables->sign_words[3];
+        auto kern = signs ? dequantize_v5_kernel<PW, BF16, true> : dequantize_v5_kernel<PW, BF16, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t chunks = (a.nblocks + 31) / 32;
+        const int64_t want = (chunks + kW5 - 1) / kW5;
+        const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
+        kern<<<(unsigned)(grid > 0 ? grid : 1), kW5 * 32, smem, st>>>(static_cast<const uint8_t *>(a.codes),
+                                                                     a.norms, a.nblocks, *a.tables, a.tmap_out32);
+        return cudaGetLastError();
+    }
+}
+
+template <int D, int PW, bool BF16>
+static cudaError_t launch_qjl6(const QuantArgs &a, cudaStream_t st)
+{
+    if constexpr (D != 128) {
+        return cudaErrorNotSupported;
+    } else {
+        if (!a.has_tmap_v || a.tables->sat_cells <= 0) return cudaErrorNotSupported;
+        if ((size_t)kGroups6 * qjl_v6_nacc(a.m) * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
+        const size_t smem = qjl_v6_smem(a.m, *a.tables);
+        if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+        const bool signs = a.tables->sign_words[0] | a.tables->sign_words[1] | a.tables->sign_words[2] |
+                           a.tables->sign_words[3];
+        auto kern = signs ? qjl_v6_quant_kernel<PW, BF16, true> : qjl_v6_quant_kernel<PW, BF16, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t tiles = (a.nblocks + 127) / 128;
+        const int64_t want = (tiles + kGroups6 - 1) / kGroups6;
+        const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
+        kern<<<(unsigned)(grid > 0 ? grid : 1), kW6 * 32, smem, st>>>(
+            a.tmap_v, a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms, a.m,
+            static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
+        return cudaGetLastError();
+    }
+}
+
 #define RQ_CAT2(a, b, c) a##_d##b##_##c
 #define RQ_CAT(a, b, c) RQ_CAT2(a, b, c)
 #if RQ_BF16
@@ -195,6 +272,8 @@ cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_
     case PW:                                                                                              \
         if (qjl) {                                                                                        \
             {                                                                                             \
+                cudaError_t e6 = launch_qjl6<RQ_D, PW, RQ_BF16>(a, st);                                   \
+                if (e6 != cudaErrorNotSupported) return e6;                                               \
                 cudaError_t e2 = launch_qjl_v3<RQ_D, PW, RQ_BF16>(a, st);                                 \
                 if (e2 != cudaErrorNotSupported) return e2;                                               \
             }                                                                                             \
@@ -202,6 +281,10 @@ cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_
                                                              a.proj, a.qsigns, a.qnorms, a.num_sms, st);  \
             if (e != cudaErrorNotSupported) return e;                                                     \
             return launch_q<RQ_D, PW, RQ_BF16, true>(a, st);                                               \
+        }                                                                                                 \
+        {                                                                                                 \
+            cudaError_t e5 = launch_q5<RQ_D, PW, RQ_BF16>(a, st);                                         \
+            if (e5 != cudaErrorNotSupported) return e5;                                                   \
         }                                                                                                 \
         return launch_q2<RQ_D, PW, RQ_BF16>(a, st);
     switch (a.pw) {
@@ -213,8 +296,12 @@ cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_
 
 cudaError_t RQ_CAT(launch_dequantize, RQ_D, RQ_DT)(const DequantArgs &a, cudaStream_t st)
 {
-#define RQ_CASE(PW) \
-    case PW: return launch_dq2<RQ_D, PW, RQ_BF16>(a, st);
+#define RQ_CASE(PW)                                                                                       \
+    case PW: {                                                                                            \
+        cudaError_t e5 = launch_dq5<RQ_D, PW, RQ_BF16>(a, st);                                            \
+        if (e5 != cudaErrorNotSupported) return e5;                                                       \
+        return launch_dq2<RQ_D, PW, RQ_BF16>(a, st);                                                      \
+    }
     switch (a.pw) {
     RQ_CASE(1) RQ_CASE(2) RQ_CASE(3) RQ_CASE(4) RQ_CASE(5) RQ_CASE(6) RQ_CASE(7) RQ_CASE(8)
     default: return cudaErrorInvalidValue;

@@ -190,6 +190,15 @@ __device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, con
                  : "memory");
 }
 
+// 3-D tiled bulk tensor copy shared -> global (rows outside the map are clipped).
+__device__ __forceinline__ void tma_store_3d(const void *tmap, int x, int y, int z, const void *src)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N committed bulk groups still read their shared-memory source.

@@ -107,6 +107,8 @@ CASES = [
     (128, 2, L.RQ_CODES_PACKED, torch.float16, 0),
     (128, 1, L.RQ_CODES_PACKED, torch.bfloat16, 1),
     (128, 8, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (128, 4, L.RQ_CODES_INT8, torch.float16, 1),
+    (128, 6, L.RQ_CODES_PACKED, torch.bfloat16, 0),
     (64, 4, L.RQ_CODES_PACKED, torch.bfloat16, 1),
     (64, 3, L.RQ_CODES_INT8, torch.float16, 1),
     (256, 2, L.RQ_CODES_PACKED, torch.bfloat16, 1),
@@ -230,25 +232,40 @@ def test_sketch_keys(d, m):
     assert np.array_equal(norms.cpu().numpy().view(np.uint16), O.vec_norms(k16, O.BF16, d))
 
 
-@pytest.mark.parametrize("d,bits,m", [(128, 4, 128), (128, 3, 128), (128, 5, 128), (256, 2, 256), (512, 2, 512)])
-def test_quantize_qjl_residual(d, bits, m):
+QJL_CASES = [
+    # d, bits, m, layout, dtype, signs
+    (128, 4, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (128, 3, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (128, 5, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (128, 1, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (128, 2, 40, L.RQ_CODES_PACKED, torch.float16, 0),
+    (128, 6, 64, L.RQ_CODES_INT8, torch.float16, 1),
+    (256, 2, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (256, 4, 72, L.RQ_CODES_PACKED, torch.float16, 1),
+    (512, 2, 512, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+]
+
+
+@pytest.mark.parametrize("d,bits,m,layout,dtype,signs", QJL_CASES)
+def test_quantize_qjl_residual(d, bits, m, layout, dtype, signs):
     nblocks = 2 * 128 + 11
-    x = synth.student_t_outliers(1, nblocks * d, seed=7 + d, device=DEV).reshape(-1)
+    x = synth.student_t_outliers(1, nblocks * d, seed=7 + d + m, dtype=dtype, device=DEV).reshape(-1)
     cent = L.rq_lloyd_max(bits)
     S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
     L.qjl_make_projection(2, m, d, S)
-    codes = torch.empty(L.rq_code_bytes(x.numel(), d, bits, L.RQ_CODES_PACKED), dtype=torch.uint8, device=DEV)
+    codes = torch.empty(L.rq_code_bytes(x.numel(), d, bits, layout), dtype=torch.uint8, device=DEV)
     norms = torch.empty(nblocks, dtype=torch.int16, device=DEV)
     qs = torch.empty(nblocks * m // 8, dtype=torch.uint8, device=DEV)
     qn = torch.empty(nblocks, dtype=torch.int16, device=DEV)
-    L.rq_quantize_qjl(x, d, bits, L.RQ_CODES_PACKED, 1, 1, cent, m, S, codes, norms, qs, qn)
+    L.rq_quantize_qjl(x, d, bits, layout, signs, 1, cent, m, S, codes, norms, qs, qn)
     torch.cuda.synchronize()
     x16 = u16(x)
-    s = O.sign_diagonal(1, d)
-    oc, on, _, _ = O.quantize(x16, O.BF16, d, bits, O.PACKED, s, cent)
-    check_codes(codes.cpu().numpy(), oc, x16, O.BF16, d, bits, O.PACKED, s, cent)
+    dt = dt_code(dtype)
+    s = O.sign_diagonal(1, d) if signs else None
+    oc, on, _, _ = O.quantize(x16, dt, d, bits, layout, s, cent)
+    check_codes(codes.cpu().numpy(), oc, x16, dt, d, bits, layout, s, cent)
     assert np.array_equal(norms.cpu().numpy().view(np.uint16), on)
-    r_bf, rn = O.residual(x16, O.BF16, oc, on, d, bits, O.PACKED, s, cent)
+    r_bf, rn = O.residual(x16, dt, oc, on, d, bits, layout, s, cent)
     assert np.array_equal(qn.cpu().numpy().view(np.uint16), rn)
     osg, p = O.sketch(r_bf, O.BF16, d, m, u16(S), want_p=True)
     check_signs(qs.cpu().numpy(), osg, p, nblocks, m)

@@ -130,3 +130,15 @@ def test_score_workspace_size_and_check():
         L.qjl_score(FakeTensor(0x40000), 8, 32, 256, 256, FakeTensor(0x50000), FakeTensor(0x60000),
                     FakeTensor(0x70000), 1000, FakeTensor(0x80000), small, stream=0)
     assert e.value.status == -3
+
+
+def test_table_cache_miss_and_hit_paths():
+    """Valid calls build (miss) and then reuse (hit) the per-call tables; with
+    no GPU visible the call stops right after, at the device query."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible: the call would launch")
+    for bits in (3, 4, 3, 4, 2, 5, 6, 7, 1, 8, 3):          # more configurations than cache slots
+        with pytest.raises(L.RQError) as e:
+            _q(FakeTensor(0x30000), bits=bits)
+        assert e.value.status == -5
