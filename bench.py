@@ -147,6 +147,12 @@ def job_rate(units_per_rank_step, world, steps, max_ms):
     return units_per_rank_step * world * steps / (max_ms * 1e-3)
 
 
+# DRAM bytes (read + write) of one 4-bit launch of each headline kernel, measured with
+# ncu (--set full) on the 8192 x 8192 weight; scaled to a workload by element count.
+# Writes still dirty in L2 when a kernel ends are not in the DRAM count.
+NCU_DRAM_BYTES_8192SQ = {"qjl_v6": 134.51e6 + 24.67e6, "dequantize_v5": 34.65e6 + 75.72e6}
+
+
 def alg_bytes_quant(n, bits):
     return n * 2 + n * bits / 8 + 2 * n / D
 
@@ -241,8 +247,10 @@ def run_device(args, rank, world):
     dq_ms = [statistics.mean(kern_ms[s][2 * i + 1] for s in range(args.steps)) for i in range(len(BITS))]
     if sum(q_ms) >= sum(dq_ms):
         dom, alg, ms = "qjl_v6_quant_kernel<b,bf16,signs> (d=128)", sum(alg_bytes_quant_qjl(n, b) for b in BITS), sum(q_ms)
+        traffic = NCU_DRAM_BYTES_8192SQ["qjl_v6"] * n / 8192 ** 2
     else:
         dom, alg, ms = "dequantize_v5_kernel<b,bf16,signs> (d=128)", sum(alg_bytes_dequant(n, b) for b in BITS), sum(dq_ms)
+        traffic = NCU_DRAM_BYTES_8192SQ["dequantize_v5"] * n / 8192 ** 2
     achieved = alg / (ms * 1e-3) / 1e9
     per_kernel = {f"quantize_qjl_b{b}_ms": round(q, 4) for b, q in zip(BITS, q_ms)}
     per_kernel.update({f"dequantize_b{b}_ms": round(q, 4) for b, q in zip(BITS, dq_ms)})
@@ -290,7 +298,11 @@ def run_device(args, rank, world):
                    "l2": "flushed (256 MB read) before every kernel; step time = sum of kernel times", "parallelism": f"replicas x{world}"},
         "pct_hbm_peak": round(100 * achieved / hbm, 1),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "peak_source": src, "traffic": None,
+                     "frac": round(achieved / hbm, 4), "peak_source": src, "traffic": round(traffic),
+                     "traffic_note": "ncu dram read+write of the 4-bit launch on the 8192^2 weight, scaled by "
+                                     "elements; per launch (achieved covers the 3-bit, 4-bit and 5-bit launches)",
+                     "alg_bytes_per_launch_4bit": round(alg_bytes_quant_qjl(n, 4) if dom.startswith("qjl")
+                                                        else alg_bytes_dequant(n, 4)),
                      "alg_bytes_per_step": alg},
         "kernels": per_kernel,
         "quantize_dequantize_only": qd,
