@@ -102,7 +102,9 @@ __device__ __forceinline__ void store_half64(uint32_t row_base, int blk, uint32_
 }
 
 // Canonical pairwise sum of squares of the whole block: the lane's 64-value
-// half (aligned 8-leaf subtrees), then the two halves added.
+// part (aligned 8-leaf subtrees), then the parts of the block's LANES lanes
+// (lane strides STRIDE, 2*STRIDE, ...: adjacent 64-value parts first).
+template <int LANES = 2, int STRIDE = 16>
 __device__ __forceinline__ float sumsq_half64(const float2 *P)
 {
     float2 t[4];
@@ -121,12 +123,17 @@ __device__ __forceinline__ float sumsq_half64(const float2 *P)
     t[0] = __fadd2_rn(t[0], t[1]);
     t[2] = __fadd2_rn(t[2], t[3]);
     t[0] = __fadd2_rn(t[0], t[2]);
-    const float half = __fadd_rn(t[0].x, t[0].y);
-    return __fadd_rn(half, __shfl_xor_sync(0xffffffffu, half, 16));
+    float part = __fadd_rn(t[0].x, t[0].y);
+#pragma unroll
+    for (int l = 1; l < LANES; l *= 2) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, STRIDE * l));
+    return part;
 }
 
-// Stages h = 1..32 in the lane, h = 64 across the lane pair (lane ^ 16).
-__device__ __forceinline__ void fwht_half64(float2 *P, bool upper)
+// Stages h = 1..32 in the lane, then h = 64, 128, ... across the block's
+// LANES lanes (partner lane ^ STRIDE*l for stage 64*l); `q` = the lane's
+// 64-value part index within the block.
+template <int LANES = 2, int STRIDE = 16>
+__device__ __forceinline__ void fwht_half64(float2 *P, int q)
 {
     const float2 m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
@@ -145,14 +152,17 @@ __device__ __forceinline__ void fwht_half64(float2 *P, bool upper)
         P[i].x = __fadd_rn(a, b);
         P[i].y = __fsub_rn(a, b);
     }
-    const float sg = upper ? -1.0f : 1.0f;              // stage h = 64
-    const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        float2 o;
-        o.x = __shfl_xor_sync(0xffffffffu, P[i].x, 16);
-        o.y = __shfl_xor_sync(0xffffffffu, P[i].y, 16);
-        P[i] = __ffma2_rn(P[i], sg2, o);                // lower: mine + other; upper: other - mine
+    for (int l = 1; l < LANES; l *= 2) {                // stages h = 64 l
+        const float sg = (q & l) ? -1.0f : 1.0f;
+        const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            float2 o;
+            o.x = __shfl_xor_sync(0xffffffffu, P[i].x, STRIDE * l);
+            o.y = __shfl_xor_sync(0xffffffffu, P[i].y, STRIDE * l);
+            P[i] = __ffma2_rn(P[i], sg2, o);            // lower: mine + other; upper: other - mine
+        }
     }
 }
 
@@ -300,7 +310,7 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
         float2 P[32];
         load_half64<BF16, SIGNS>(rbase, blk_row, pmh, P, false);
         const float n32 = __fsqrt_rn(sumsq_half64(P));
-        fwht_half64(P, hf != 0);
+        fwht_half64(P, hf);
         const float inv = n32 > 0.0f ? __frcp_rn(n32) : 0.0f;
         uint32_t w[2 * PW];
         codes_half64<PW>(P, inv, G, w);
@@ -314,7 +324,7 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
             if (!mbar_wait(&mma_done[pslot], (uint32_t)(((k - 1) / kNSG6) & 1))) ok = false;
             else if (tile_of(k - 1 + kNSG6) < t1) load_tile(k - 1 + kNSG6);
         }
-        fwht_half64(P, hf != 0);
+        fwht_half64(P, hf);
         const float nsc = -__fmul_rn(h16_to_f32(n16), 1.0f / 128.0f);
         residual_half64<BF16, SIGNS>(rbase, blk_row, pmh, make_float2(nsc, nsc), P);
         const float rn32 = __fsqrt_rn(sumsq_half64(P));

@@ -205,6 +205,43 @@ def test_weight_4096x4096_sampled_full_size():
         assert np.array_equal(u16(out.view(-1, 128)[torch.from_numpy(blocks).to(DEV)]), oo)
 
 
+LLAMA7B_LINEARS = [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]   # q, k, v, o, gate, up, down
+
+
+def test_llama7b_32_layers_one_call_sampled():
+    """All linears of 32 Llama-7B-shaped layers (6.48e9 bf16 values, 50.6M
+    blocks, 13 GB) quantized (4-bit, d = 128, seeded signs) and dequantized
+    with one call each -- the largest input of the workloads -- and 2048
+    blocks sampled over every layer and matrix checked against the oracle."""
+    sizes = [r * c for r, c in LLAMA7B_LINEARS] * 32
+    n = sum(sizes)
+    x = torch.empty(n, dtype=torch.bfloat16, device=DEV)
+    off = 0
+    for i, (r, c) in enumerate(LLAMA7B_LINEARS * 32):
+        x[off:off + r * c] = synth.llama_linear(r, c, seed=1000 + i, device=DEV).reshape(-1)
+        off += r * c
+    bits, seed = 4, 11
+    cent = L.rq_lloyd_max(bits)
+    codes, norms = run_quant(x, 128, bits, L.RQ_CODES_PACKED, 1, seed, cent)
+    out = torch.empty_like(x)
+    L.rq_dequantize(codes, norms, n, 128, bits, L.RQ_CODES_PACKED, 1, seed, cent, out)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    nb = n // 128
+    blocks = np.unique(np.concatenate([rng.choice(nb, 2040, replace=False), [0, 1, nb - 2, nb - 1]]))
+    idx = torch.from_numpy(blocks).to(DEV)
+    xs = u16(x.view(-1, 128)[idx])
+    s = O.sign_diagonal(seed, 128)
+    gc = codes.view(-1, 64)[idx].cpu().numpy().reshape(-1)
+    oc, on, _, _ = O.quantize(xs, O.BF16, 128, bits, O.PACKED, s, cent)
+    check_codes(gc, oc, xs, O.BF16, 128, bits, O.PACKED, s, cent)
+    assert np.array_equal(norms.view(torch.int16).cpu().numpy().view(np.uint16)[blocks], on)
+    oo, _ = O.dequantize(oc, on, 128, bits, O.PACKED, s, cent, O.BF16)
+    assert np.array_equal(u16(out.view(-1, 128)[idx]), oo)
+    del x, out, codes, norms
+    torch.cuda.empty_cache()
+
+
 # ------------------------------------------------------------------ QJL
 
 @pytest.mark.parametrize("m,d,dtype", [(128, 128, torch.bfloat16), (256, 128, torch.bfloat16),
@@ -242,6 +279,7 @@ QJL_CASES = [
     (128, 6, 64, L.RQ_CODES_INT8, torch.float16, 1),
     (256, 2, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1),
     (256, 4, 72, L.RQ_CODES_PACKED, torch.float16, 1),
+    (256, 3, 128, L.RQ_CODES_INT8, torch.bfloat16, 0),
     (512, 2, 512, L.RQ_CODES_PACKED, torch.bfloat16, 1),
 ]
 
