@@ -20,7 +20,7 @@
 // Memory.  The 128-value rows of a 32-block chunk arrive by 3-D TMA
 // ({64 values, 2 halves, 32 blocks}, 128-byte swizzle: lane r reads row r
 // without bank conflicts); every warp runs its own ring of chunks, with no
-// barrier shared with other warps.  (The fused quantize+QJL kernel for d = 128
+// barrier shared with other warps; twelve warps per CTA at 168 registers.  (The fused quantize+QJL kernel for d = 128
 // is in rq_v6.cuh: with a whole block per thread its loop outgrew the
 // instruction cache, so it splits each block over two lanes.)
 #pragma once
@@ -31,8 +31,8 @@
 
 namespace rq {
 
-constexpr int kW5 = 8;                      // compute warps per CTA
-constexpr int kNSW5 = 3;                    // per-warp ring depth (quantize)
+constexpr int kW5 = 12;                     // warps per CTA (168 registers each)
+constexpr int kNSW5 = 2;                    // per-warp ring depth (quantize)
 constexpr uint32_t kChunkBytes5 = 32u * 256u;   // 32 rows x 2 halves x 128 B
 
 __device__ __forceinline__ float fma_sat(float a, float b, float c)
@@ -331,7 +331,7 @@ __host__ __device__ inline int cent_copies5(int levels) { return levels <= 32 ? 
 
 __host__ __device__ inline size_t dequantize_v5_smem(int pw, int levels)
 {
-    return 1024 + (size_t)kW5 * 2 * kChunkBytes5 + (size_t)kW5 * kNSD5 * 512 * pw +
+    return 1024 + (size_t)kW5 * kChunkBytes5 + (size_t)kW5 * kNSD5 * 512 * pw +
            (size_t)levels * cent_copies5(levels) * 4 + 256 + 8 * kW5 * kNSD5;
 }
 
@@ -344,8 +344,8 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
     constexpr uint32_t RING = 512u * PW;          // one chunk's codes
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *outb = base;                                         // kW5 x 2 staging chunks
-    uint8_t *cring = outb + (size_t)kW5 * 2 * kChunkBytes5;       // kW5 x kNSD5 code chunks
+    uint8_t *outb = base;                                         // kW5 staging chunks
+    uint8_t *cring = outb + (size_t)kW5 * kChunkBytes5;           // kW5 x kNSD5 code chunks
     float *cent = reinterpret_cast<float *>(cring + (size_t)kW5 * kNSD5 * RING);
     const int copies = cent_copies5(T.levels);
     uint32_t *pmask = reinterpret_cast<uint32_t *>(cent + T.levels * copies);
@@ -365,7 +365,7 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
     __syncthreads();
 
     uint8_t *wring = cring + (size_t)warp * kNSD5 * RING;
-    uint8_t *wout = outb + (size_t)warp * 2 * kChunkBytes5;
+    uint8_t *wout = outb + (size_t)warp * kChunkBytes5;
     uint64_t *wfull = full + warp * kNSD5;
     auto issue = [&](int64_t j, int s) {
         const int64_t nb = nblocks - j * 32 < 32 ? nblocks - j * 32 : 32;
@@ -420,8 +420,8 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
         const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
         for (int i = 0; i < 64; ++i) P[i] = __fmul2_rn(P[i], sc2);
-        uint8_t *ob = wout + (size_t)(k & 1) * kChunkBytes5;
-        if (lane == 0) bulk_wait_read<1>();              // the store from two chunks ago has left ob
+        uint8_t *ob = wout;
+        if (lane == 0) bulk_wait_read<0>();              // the previous chunk's store has left ob
         __syncwarp();
         store_row128<BF16, SIGNS>(smem_u32(ob), kChunkBytes5 / 2, lane, pm, P);
         fence_proxy_async_smem();
