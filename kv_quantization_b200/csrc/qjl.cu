@@ -11,7 +11,7 @@
 
 #include "rq_common.cuh"
 #include "rq_kernels.h"
-#include "qjl_score_v3.cuh"
+#include "qjl_score_v4.cuh"
 
 namespace rq {
 
@@ -187,11 +187,22 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
         a.q, a.nq, a.d, a.m, static_cast<const uint16_t *>(a.proj), a.proj_bf16, *a.tables, TWO, wsB, wsN);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    const int64_t items = a.G * ((a.T + 127) / 128);
+    const int64_t grid = items < (int64_t)a.num_sms ? items : (int64_t)a.num_sms;
+    // eight producer warps (qjl_score_v4.cuh) with the deepest chunk ring that fits
+    for (int ring = kSc4MaxRing; ring >= 3; --ring) {
+        const size_t smem4 = sc4_smem(a.nq, a.d, a.m, TWO, PW, ring);
+        if (smem4 > kMaxSmemPerBlock) continue;
+        auto kern4 = score_v4_kernel<PW, TWO>;
+        e = cudaFuncSetAttribute(kern4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem4);
+        if (e != cudaSuccess) return e;
+        kern4<<<(unsigned)(grid > 0 ? grid : 1), kSc4Threads, smem4, st>>>(
+            wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms, a.T, a.G, a.codes, a.norms, *a.tables, a.scores, ring);
+        return cudaGetLastError();
+    }
     auto kern = score_v3_kernel<PW, TWO>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t items = a.G * ((a.T + 127) / 128);
-    const int64_t grid = items < (int64_t)a.num_sms ? items : (int64_t)a.num_sms;
     kern<<<(unsigned)(grid > 0 ? grid : 1), kSc3Threads, smem, st>>>(wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms,
                                                                      a.T, a.G, a.codes, a.norms, *a.tables, a.scores);
     return cudaGetLastError();

@@ -15,7 +15,8 @@
 // straight into the tensor-core A layout); a tile's rows are block =
 // 16 * warp + (lane mod 16) and its two halves sit in the two 64-column
 // regions, so a quarter-warp's 16-byte loads touch eight different bank
-// groups.  The residual overwrites the tile in place as the bf16 A operand,
+// groups.  The residual r' = s * r overwrites the tile in place as the bf16 A
+// operand (the sign diagonal is folded into the staged projection S' = S diag(s)),
 // the last of the group's eight warps to finish issues the sketch MMA
 // (P = R S^T into TMEM), the sign epilogue of a tile runs after the next tile
 // is computed, and the group's first warp refills a stage in the middle of the
@@ -29,6 +30,32 @@ constexpr int kW6 = 16;                       // warps per CTA
 constexpr int kGroups6 = 2;                   // groups of eight warps
 constexpr int kNSG6 = 2;                      // tile ring depth per group
 constexpr uint32_t kTileBytes6 = 128u * 256u;  // 128 blocks x 2 regions x 128 B
+
+// Stage S' = S diag(s) (the sign diagonal folded into the projection's
+// columns: a bf16 sign flip is exact, so P = r' S'^T = r S^T bit for bit with
+// r' = s * r the residual before its final sign flip) in the tcgen05 B layout.
+template <int D, bool SIGNS>
+__device__ __forceinline__ void stage_projection_signed(const uint16_t *__restrict__ proj, uint8_t *s_S, int m,
+                                                        int m16, const QuantTables &T)
+{
+    for (int idx = threadIdx.x; idx < m16 * (D / 8); idx += blockDim.x) {
+        const int i = idx / (D / 8), c = idx % (D / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i < m) v = __ldg(reinterpret_cast<const uint4 *>(proj + (size_t)i * D) + c);
+        if constexpr (SIGNS) {
+            uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 8 * c + 2 * e;            // values j, j + 1 of the row
+                const uint32_t b0 = (T.sign_words[j >> 5] >> (j & 31)) & 1u;
+                const uint32_t b1 = (T.sign_words[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u;
+                x[e] ^= (b0 << 15) | (b1 << 31);
+            }
+            v = make_uint4(x[0], x[1], x[2], x[3]);
+        }
+        *reinterpret_cast<uint4 *>(s_S + (size_t)(c >> 3) * m16 * 128 + sw128_offset(i, c & 7)) = v;
+    }
+}
 
 template <bool BF16, bool SIGNS>
 __device__ __forceinline__ void load_half64(uint32_t row_base, int blk, uint32_t pmask_half, float2 *P, bool fresh)
@@ -255,7 +282,7 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
     if (lw == 0 && lane == 0)
         for (int k = 0; k < kNSG6; ++k)
             if (tile_of(k) < t1) load_tile(k);
-    stage_projection_d<128>(proj, s_S, m, m16);
+    stage_projection_signed<128, SIGNS>(proj, s_S, m, m16, T);
     setup_sat_lut16(T, reinterpret_cast<uint4 *>(lutb));
     setup_pair_masks(T, pmask, 128);
     if (warp == 0) tmem_alloc(tmem_slot, ncols);
@@ -329,7 +356,7 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
         residual_half64<BF16, SIGNS>(rbase, blk_row, pmh, make_float2(nsc, nsc), P);
         const float rn32 = __fsqrt_rn(sumsq_half64(P));
         if (valid && hf == 0) qnorms[blk] = norm_to_h16(rn32);
-        store_half64<SIGNS>(rbase, blk_row, pmh, P);
+        store_half64<false>(rbase, blk_row, pmh, P);     // r' (signs live in S')
         fence_proxy_async_smem();
         if (k >= 1) epilogue(k - 1);
         if (!__all_sync(0xffffffffu, ok)) break;

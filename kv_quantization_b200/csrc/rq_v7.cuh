@@ -6,7 +6,8 @@
 // stages h = 1..32 run in the lane, h = 64 and h = 128 across lanes (xor 8,
 // xor 16), the pairwise norm adds the parts in the same order.  Sixteen warps
 // cover one 128-block tile, whose four 64-column regions are the tcgen05 A
-// operand (K = 256) after the residual overwrites them in place.
+// operand (K = 256) after the residual r' = s * r overwrites them in place
+// (the sign diagonal is folded into the staged projection, as in rq_v6.cuh).
 //
 // The projection S (m x 256 bf16) takes up to 128 KB of shared memory, which
 // leaves room for one tile: the tile's buffer is refilled as soon as the MMA
@@ -78,7 +79,7 @@ qjl_v7_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
     }
     __syncthreads();
     if (threadIdx.x == 0 && t0 < t1) load_tile(t0);
-    stage_projection_d<256>(proj, s_S, m, m16);
+    stage_projection_signed<256, SIGNS>(proj, s_S, m, m16, T);
     setup_sat_lut16(T, reinterpret_cast<uint4 *>(lutb));
     setup_pair_masks(T, pmask, 256);
     if (warp == 0) tmem_alloc(tmem_slot, ncols);
@@ -146,7 +147,7 @@ qjl_v7_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
         residual_half64<BF16, SIGNS>(rbase, blk_row, pmq, make_float2(nsc, nsc), P);
         const float rn32 = __fsqrt_rn(sumsq_half64<4, 8>(P));
         if (valid && q == 0) qnorms[blk] = norm_to_h16(rn32);
-        store_half64<SIGNS>(rbase, blk_row, pmq, P);
+        store_half64<false>(rbase, blk_row, pmq, P);     // r' (signs live in S')
         fence_proxy_async_smem();
         if (k >= 1) epilogue(k - 1);
         if (!__all_sync(0xffffffffu, ok)) break;
