@@ -179,10 +179,10 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
     const size_t rows = (size_t)a.G * a.nq;
     float *wsN = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.workspace) +
                                            ((rows * sc2_kb(a.d, a.m, TWO) * 2 + 255) & ~(size_t)255));
-    const size_t psmem = ((size_t)2 * kSc2PrologueQ * a.d + kSc2PrologueQ) * sizeof(float);
+    const size_t psmem = sc2_prologue_smem(a.d);
     cudaError_t e = cudaFuncSetAttribute(score_v2_prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess) return e;
-    const unsigned zsl = (unsigned)((sc2_m64(a.m) + 31) / 32);       // 32 S q outputs per CTA
+    const unsigned zsl = (unsigned)((sc2_m64(a.m) + kSc2PrologueOut - 1) / kSc2PrologueOut);   // 16 S q outputs per CTA
     score_v2_prologue<<<dim3((unsigned)a.G, (unsigned)((a.nq + kSc2PrologueQ - 1) / kSc2PrologueQ), zsl), 256, psmem, st>>>(
         a.q, a.nq, a.d, a.m, static_cast<const uint16_t *>(a.proj), a.proj_bf16, *a.tables, TWO, wsB, wsN);
     e = cudaGetLastError();

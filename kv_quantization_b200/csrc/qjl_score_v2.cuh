@@ -65,15 +65,24 @@ __host__ __device__ inline size_t sc2_smem(int nq, int d, int m, bool two, int p
 // butterfly in shared memory) and S q (fp32, each thread one row of S against
 // all queries), both scaled by 1/||q|| and rounded to fp16, plus ||q|| itself.
 constexpr int kSc2PrologueQ = 32;
+constexpr int kSc2PrologueOut = 16;                 // S q outputs per CTA (16 rows x 16 query pairs = 256 threads)
+
+// Shared memory of score_v2_prologue: [32][d] signed copy (rotated in place),
+// [d][32] transposed raw copy (the S q operand), [32] inverse norms.
+__host__ __device__ inline size_t sc2_prologue_smem(int d)
+{
+    return ((size_t)2 * kSc2PrologueQ * d + kSc2PrologueQ) * sizeof(float);
+}
 
 __global__ void __launch_bounds__(256)
 score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const uint16_t *__restrict__ proj,
                   bool proj_bf16, const __grid_constant__ QuantTables T, bool two, uint16_t *__restrict__ wsB,
                   float *__restrict__ wsN)
 {
-    extern __shared__ float pq[];                  // [32][d] raw, [32][d] rotated, [32] inverse norms
-    float *pr = pq + kSc2PrologueQ * d;
-    float *pinv = pr + kSc2PrologueQ * d;
+    extern __shared__ float pq[];
+    float *pr = pq;                                 // [32][d]: D q, rotated in place to H D q
+    float *pt = pr + kSc2PrologueQ * d;             // [d][32]: q, transposed
+    float *pinv = pt + kSc2PrologueQ * d;           // [32] 1 / ||q||
     const int64_t g = blockIdx.x;
     const int q0 = blockIdx.y * kSc2PrologueQ;
     const int zs = blockIdx.z, nz = gridDim.z;        // slice of the S q outputs (z = 0 also rotates)
@@ -83,13 +92,13 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
         const int qi = idx / d, j = idx % d;
         float v = 0.0f;
         if (qi < nqc) v = __uint_as_float((uint32_t)q[((int64_t)g * nq + q0 + qi) * d + j] << 16);
-        pq[idx] = v;
+        pt[j * kSc2PrologueQ + qi] = v;
         pr[idx] = __uint_as_float(__float_as_uint(v) ^ sign_mask(T.sign_words, j));
     }
     __syncthreads();
     for (int qi = warp; qi < kSc2PrologueQ; qi += blockDim.x / 32) {
         float sum = 0.0f;
-        for (int j = lane; j < d; j += 32) sum = __fmaf_rn(pq[qi * d + j], pq[qi * d + j], sum);
+        for (int j = lane; j < d; j += 32) sum = __fmaf_rn(pr[qi * d + j], pr[qi * d + j], sum);
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane == 0) {
             const float qn = sqrtf(sum);
@@ -116,12 +125,11 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
             const int qi = idx / d, j = idx % d;
             wsB[((int64_t)g * nq + q0 + qi) * kb + j] = __half_as_ushort(__float2half_rn(pr[idx] * pinv[qi]));
         }
-    const int per = (sc2_m64(m) + nz - 1) / nz;
-    const int i_lo = zs * per, i_hi = min(sc2_m64(m), i_lo + per);
-    for (int i = i_lo + tid; i < i_hi; i += blockDim.x) {
-        float acc[kSc2PrologueQ];
-#pragma unroll
-        for (int qi = 0; qi < kSc2PrologueQ; ++qi) acc[qi] = 0.0f;
+    // S q: output row i = i_lo + tid / 16 of this slice, queries 2 (tid % 16) and 2 (tid % 16) + 1
+    const int per = (sc2_m64(m) + nz - 1) / nz;       // <= kSc2PrologueOut (launch)
+    const int i = zs * per + tid / 16, qp = 2 * (tid % 16);
+    if (tid / 16 < per && i < sc2_m64(m)) {
+        float acc0 = 0.0f, acc1 = 0.0f;
         if (i < m) {
             const uint4 *Srow = reinterpret_cast<const uint4 *>(proj + (int64_t)i * d);
             for (int j8 = 0; j8 < d / 8; ++j8) {
@@ -131,14 +139,17 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
                 for (int e = 0; e < 8; ++e) {
                     const uint16_t h = (uint16_t)(ws4[e >> 1] >> (16 * (e & 1)));
                     const float sv = proj_bf16 ? __uint_as_float((uint32_t)h << 16) : h16_to_f32(h);
-                    const int j = j8 * 8 + e;
-#pragma unroll
-                    for (int qi = 0; qi < kSc2PrologueQ; ++qi) acc[qi] = __fmaf_rn(sv, pq[qi * d + j], acc[qi]);
+                    const float2 qv = *reinterpret_cast<const float2 *>(pt + (j8 * 8 + e) * kSc2PrologueQ + qp);
+                    acc0 = __fmaf_rn(sv, qv.x, acc0);
+                    acc1 = __fmaf_rn(sv, qv.y, acc1);
                 }
             }
         }
-        for (int qi = 0; qi < nqc; ++qi)
-            wsB[((int64_t)g * nq + q0 + qi) * kb + off + i] = __half_as_ushort(__float2half_rn(acc[qi] * pinv[qi]));
+        if (qp < nqc)
+            wsB[((int64_t)g * nq + q0 + qp) * kb + off + i] = __half_as_ushort(__float2half_rn(acc0 * pinv[qp]));
+        if (qp + 1 < nqc)
+            wsB[((int64_t)g * nq + q0 + qp + 1) * kb + off + i] =
+                __half_as_ushort(__float2half_rn(acc1 * pinv[qp + 1]));
     }
 }
 
