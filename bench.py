@@ -369,7 +369,8 @@ def secondary_scores(dev, reps=5):
     out.append(_time_pair("kv 4x8x32768x128 QJL m=256",
                           lambda: rq.qjl_sketch(k, d, m, S, signs, kn),
                           lambda: rq.qjl_score(q, G, nq, d, m, S, signs, kn, T, scores, ws), G * T,
-                          2 * m * d * G * T, k.numel() * 2 + signs.numel() + kn.numel() * 2, reps))
+                          2 * m * d * G * T, k.numel() * 2 + signs.numel() + kn.numel() * 2, reps,
+                          score_bytes=signs.numel() + kn.numel() * 2 + 4 * G * nq * T))
     del k, signs, kn, scores, ws
     # TurboQuant-style 3-bit keys, head_dim 256: 2-bit + QJL m = d
     G, T, d, bits = 8, 131072, 256, 2
@@ -391,11 +392,34 @@ def secondary_scores(dev, reps=5):
                           lambda: rq.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms,
                                                bits=bits, layout=rq.RQ_CODES_PACKED, use_signs=1, sign_seed=4,
                                                centroids=cent),
-                          G * T, 2 * m * d * G * T, k.numel() * 2 + codes.numel() + qs.numel() + 4 * G * T, reps))
+                          G * T, 2 * m * d * G * T, k.numel() * 2 + codes.numel() + qs.numel() + 4 * G * T, reps,
+                          score_bytes=codes.numel() + qs.numel() + 4 * G * T + 4 * G * nq * T))
+    del k, codes, norms, qs, qn, scores, ws
+    # the same at head_dim 512 (m = d = 512)
+    G, T, d, bits = 8, 131072, 512, 2
+    m = d
+    k = synth.normal((G, T, d), seed=8, device=dev).reshape(-1)
+    S = torch.empty(m, d, dtype=torch.bfloat16, device=dev)
+    rq.qjl_make_projection(9, m, d, S)
+    codes = torch.empty(rq.rq_code_bytes(k.numel(), d, bits, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev)
+    norms = torch.empty(G * T, dtype=torch.int16, device=dev)
+    qs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=dev)
+    qn = torch.empty(G * T, dtype=torch.int16, device=dev)
+    q = synth.normal((G, nq, d), seed=10, device=dev)
+    scores = torch.empty(G, nq, T, dtype=torch.float32, device=dev)
+    ws = torch.empty(rq.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=dev)
+    out.append(_time_pair("keys 131072x8 d=512 2-bit+QJL m=d",
+                          lambda: rq.rq_quantize_qjl(k, d, bits, rq.RQ_CODES_PACKED, 1, 4, cent, m, S, codes, norms,
+                                                     qs, qn),
+                          lambda: rq.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms,
+                                               bits=bits, layout=rq.RQ_CODES_PACKED, use_signs=1, sign_seed=4,
+                                               centroids=cent),
+                          G * T, 2 * m * d * G * T, k.numel() * 2 + codes.numel() + qs.numel() + 4 * G * T, reps,
+                          score_bytes=codes.numel() + qs.numel() + 4 * G * T + 4 * G * nq * T))
     return out
 
 
-def _time_pair(name, prep, score, tokens, prep_flops, prep_bytes, reps=5):
+def _time_pair(name, prep, score, tokens, prep_flops, prep_bytes, reps=5, score_bytes=None):
     import torch
     prep()
     score()
@@ -415,6 +439,20 @@ def _time_pair(name, prep, score, tokens, prep_flops, prep_bytes, reps=5):
     res["score_tokens_per_s"] = round(tokens / (res["score_ms"] * 1e-3), 1)
     res["compress_gbs"] = round(prep_bytes / (res["compress_ms"] * 1e-3) / 1e9, 1)
     res["compress_tflops"] = round(prep_flops / (res["compress_ms"] * 1e-3) / 1e12, 2)
+    hbm, tf, src = peaks()
+    # compress: HBM-bound below the ridge (2 m d flops against 2 d + m/8 + ... bytes per vector)
+    ridge = tf * 1e12 / (hbm * 1e9)
+    if prep_flops / prep_bytes < ridge:
+        res["compress_roofline"] = {"bound": "hbm", "achieved": res["compress_gbs"], "peak": hbm, "unit": "GB/s",
+                                    "frac": round(res["compress_gbs"] / hbm, 4)}
+    else:
+        res["compress_roofline"] = {"bound": "tensor", "achieved": res["compress_tflops"], "peak": tf,
+                                    "unit": "TFLOP/s", "frac": round(res["compress_tflops"] / tf, 4)}
+    if score_bytes:
+        gbs = score_bytes / (res["score_ms"] * 1e-3) / 1e9
+        res["score_roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                                 "frac": round(gbs / hbm, 4),
+                                 "note": "packed keys + norms read, fp32 scores written; prologue included"}
     return res
 
 

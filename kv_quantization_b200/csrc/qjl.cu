@@ -174,7 +174,8 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
 {
     if (a.nq > 128) return cudaErrorNotSupported;
     const size_t smem = sc3_smem(a.nq, a.d, a.m, TWO, PW);
-    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+    if (smem > kMaxSmemPerBlock && sc4_smem(a.nq, a.d, a.m, TWO, PW, 2, 2, 2) > kMaxSmemPerBlock)
+        return cudaErrorNotSupported;
     uint16_t *wsB = reinterpret_cast<uint16_t *>(a.workspace);
     const size_t rows = (size_t)a.G * a.nq;
     float *wsN = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.workspace) +
@@ -189,17 +190,23 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const int64_t items = a.G * ((a.T + 127) / 128);
     const int64_t grid = items < (int64_t)a.num_sms ? items : (int64_t)a.num_sms;
-    // eight producer warps (qjl_score_v4.cuh) with the deepest chunk ring that fits
-    for (int ring = kSc4MaxRing; ring >= 3; --ring) {
-        const size_t smem4 = sc4_smem(a.nq, a.d, a.m, TWO, PW, ring);
-        if (smem4 > kMaxSmemPerBlock) continue;
-        auto kern4 = score_v4_kernel<PW, TWO>;
-        e = cudaFuncSetAttribute(kern4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem4);
-        if (e != cudaSuccess) return e;
-        kern4<<<(unsigned)(grid > 0 ? grid : 1), kSc4Threads, smem4, st>>>(
-            wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms, a.T, a.G, a.codes, a.norms, *a.tables, a.scores, ring);
-        return cudaGetLastError();
+    // eight producer warps (qjl_score_v4.cuh): the deepest configuration that fits
+    {
+        struct Cfg { int ring, nrec, slc; };
+        const Cfg cfgs[] = {{4, 3, 8}, {3, 3, 8}, {3, 2, 2}, {2, 2, 2}};
+        for (const Cfg &c : cfgs) {
+            const size_t smem4 = sc4_smem(a.nq, a.d, a.m, TWO, PW, c.ring, c.nrec, c.slc);
+            if (smem4 > kMaxSmemPerBlock) continue;
+            auto kern4 = c.nrec == 3 ? score_v4_kernel<PW, TWO, 3> : score_v4_kernel<PW, TWO, 2>;
+            e = cudaFuncSetAttribute(kern4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem4);
+            if (e != cudaSuccess) return e;
+            kern4<<<(unsigned)(grid > 0 ? grid : 1), kSc4Threads, smem4, st>>>(
+                wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms, a.T, a.G, a.codes, a.norms, *a.tables, a.scores, c.ring,
+                c.slc);
+            return cudaGetLastError();
+        }
     }
+    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;    // not reached: v4's smallest fits whenever v3 does
     auto kern = score_v3_kernel<PW, TWO>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

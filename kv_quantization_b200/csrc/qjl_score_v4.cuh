@@ -17,24 +17,26 @@ namespace rq {
 constexpr int kSc4Threads = 13 * 32;
 constexpr int kSc4MaxRing = 4;
 
-__host__ __device__ inline size_t sc4_smem(int nq, int d, int m, bool two, int pw, int ring)
+// ring: A chunks in flight; nrec: key-record tiles staged (prefetch depth nrec - 1);
+// slc: copies of the sign-byte LUT (8: conflict-free, 2: for the largest shapes)
+__host__ __device__ inline size_t sc4_smem(int nq, int d, int m, bool two, int pw, int ring, int nrec, int slc)
 {
     const int kb = sc2_kb(d, m, two), nq32 = sc2_nq16(nq);
     size_t b = 1024;
     b += (size_t)ring * kSc2ChunkBytes;                            // A ring
     b += (size_t)nq32 * kb * 2;                                    // B
-    b += (size_t)256 * 8 * 16;                                     // sign LUT
+    b += (size_t)256 * slc * 16;                                   // sign LUT
     if (two) b += pw <= 4 ? ((size_t)1 << (2 * pw)) * 32 * 4 : ((size_t)1 << pw) * 32 * 2;
-    b += 3 * (size_t)128 * sc3_row_bytes(d, m, two, pw);           // records, 3 tiles
+    b += (size_t)nrec * 128 * sc3_row_bytes(d, m, two, pw);        // staged records
     return b + 8 * (2 * kSc4MaxRing + 5) + 16;
 }
 
-template <int PW, bool TWO>
+template <int PW, bool TWO, int NREC>
 __global__ void __launch_bounds__(kSc4Threads, 1)
 score_v4_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN, int nq, int d, int m,
                 const uint8_t *__restrict__ signs, const uint16_t *__restrict__ sk_norms, int64_t T_len,
                 int64_t G, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ norms,
-                const __grid_constant__ QuantTables T, float *__restrict__ scores, int ring)
+                const __grid_constant__ QuantTables T, float *__restrict__ scores, int ring, int slc)
 {
     const int nq32 = sc2_nq16(nq), kb = sc2_kb(d, m, TWO);
     const int dreg = TWO ? d / 64 : 0;
@@ -49,10 +51,10 @@ score_v4_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
     uint8_t *sA = base;
     uint8_t *sB = sA + (size_t)ring * kSc2ChunkBytes;
     uint4 *slut = reinterpret_cast<uint4 *>(sB + (size_t)nq32 * kb * 2);
-    uint32_t *clut = reinterpret_cast<uint32_t *>(slut + 256 * 8);
+    uint32_t *clut = reinterpret_cast<uint32_t *>(slut + 256 * slc);
     const size_t clut_bytes = TWO ? (PW <= 4 ? ((size_t)1 << (2 * PW)) * 32 * 4 : ((size_t)1 << PW) * 32 * 2) : 0;
     uint8_t *srec = reinterpret_cast<uint8_t *>(clut) + clut_bytes;
-    uint64_t *a_full = reinterpret_cast<uint64_t *>(srec + 3 * 128 * rowb);
+    uint64_t *a_full = reinterpret_cast<uint64_t *>(srec + NREC * 128 * rowb);
     uint64_t *a_empty = a_full + kSc4MaxRing;
     uint64_t *acc_full = a_empty + kSc4MaxRing;
     uint64_t *acc_empty = acc_full + 2;
@@ -60,8 +62,10 @@ score_v4_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int i = tid; i < 256 * 8; i += kSc4Threads) {
-        const int byte = i >> 3;
+    const int slc_log2 = slc == 8 ? 3 : (slc == 4 ? 2 : (slc == 2 ? 1 : 0));   // slc is a power of two <= 8
+    const uint32_t slc_lane = (uint32_t)(threadIdx.x & 31) & (uint32_t)(slc - 1);
+    for (int i = tid; i < 256 * slc; i += kSc4Threads) {
+        const int byte = i >> slc_log2;
         uint32_t w[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -145,13 +149,19 @@ score_v4_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
         };
         if (it0 < it1) prefetch(it0, 0);
         cp_async_commit();
-        if (it0 + 1 < it1) prefetch(it0 + 1, 1);
-        cp_async_commit();
+        if (NREC == 3) {
+            if (it0 + 1 < it1) prefetch(it0 + 1, 1);
+            cp_async_commit();
+        }
         int64_t chunk = 0;
         for (int64_t it = it0; it < it1 && ok; ++it) {
-            const int rb = (int)((it - it0) % 3);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");   // this tile's record is in shared memory
-            if (it + 2 < it1) prefetch(it + 2, (int)((it + 2 - it0) % 3));
+            const int rb = (int)((it - it0) % NREC);
+            if constexpr (NREC == 3) {
+                asm volatile("cp.async.wait_group 1;" ::: "memory");   // this tile's record is in shared memory
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
+            if (it + NREC - 1 < it1) prefetch(it + NREC - 1, (int)((it + NREC - 1 - it0) % NREC));
             cp_async_commit();
             const int64_t t = (it % tiles_per_g) * 128 + r;
             const bool tv = t < T_len;
@@ -215,7 +225,7 @@ score_v4_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
                         for (int k = 0; k < 8; ++k) {
                             const bool live = tv && sc0 + 8 * k < m;
                             const uint32_t byte = (sb[k >> 2] >> (8 * (k & 3))) & 0xffu;
-                            const uint4 v = live ? slut[(byte << 3) + (lane & 7)] : make_uint4(0u, 0u, 0u, 0u);
+                            const uint4 v = live ? slut[(byte << slc_log2) + slc_lane] : make_uint4(0u, 0u, 0u, 0u);
                             *reinterpret_cast<uint4 *>(Ar + ((k ^ (r & 7)) << 4)) = v;
                         }
                     }

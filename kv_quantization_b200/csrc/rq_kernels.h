@@ -27,6 +27,8 @@ struct QuantArgs {
     bool has_tmap_v;
     CUtensorMap tmap_v32;      // the same view with {64, 1, 32} boxes (one warp's 32-block chunk)
     bool has_tmap_v32;
+    CUtensorMap tmap_s;        // S [m][d] 16-bit with {64, min(256, m16)} boxes (d = 512: S streamed)
+    bool has_tmap_s;
 };
 
 struct DequantArgs {

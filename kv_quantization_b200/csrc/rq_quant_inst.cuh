@@ -9,6 +9,7 @@
 #include "rq_v5.cuh"
 #include "rq_v6.cuh"
 #include "rq_v7.cuh"
+#include "rq_v8.cuh"
 #include "rq_sketch_v3.cuh"
 
 namespace rq {
@@ -234,6 +235,30 @@ static cudaError_t launch_dq5(const DequantArgs &a, cudaStream_t st)
 }
 
 template <int D, int PW, bool BF16>
+static cudaError_t launch_qjl8(const QuantArgs &a, cudaStream_t st)
+{
+    if constexpr (D != 512) {
+        return cudaErrorNotSupported;
+    } else {
+        if (!a.has_tmap_v || !a.has_tmap_s || a.tables->sat_cells <= 0 || qjl_mma_m16(a.m) > 512)
+            return cudaErrorNotSupported;
+        const size_t smem = qjl_v8_smem(*a.tables);
+        if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
+        bool signs = false;
+        for (int i = 0; i < 16; ++i) signs = signs || a.tables->sign_words[i] != 0u;
+        auto kern = signs ? qjl_v8_quant_kernel<PW, BF16, true> : qjl_v8_quant_kernel<PW, BF16, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t tiles = (a.nblocks + 127) / 128;
+        const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
+        kern<<<(unsigned)(grid > 0 ? grid : 1), kW8 * 32, smem, st>>>(
+            a.tmap_v, a.tmap_s, a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms, a.m, a.qsigns,
+            a.qnorms);
+        return cudaGetLastError();
+    }
+}
+
+template <int D, int PW, bool BF16>
 static cudaError_t launch_qjl7(const QuantArgs &a, cudaStream_t st)
 {
     if constexpr (D != 256) {
@@ -297,6 +322,8 @@ cudaError_t RQ_CAT(launch_quantize, RQ_D, RQ_DT)(const QuantArgs &a, cudaStream_
     case PW:                                                                                              \
         if (qjl) {                                                                                        \
             {                                                                                             \
+                cudaError_t e8 = launch_qjl8<RQ_D, PW, RQ_BF16>(a, st);                                   \
+                if (e8 != cudaErrorNotSupported) return e8;                                               \
                 cudaError_t e7 = launch_qjl7<RQ_D, PW, RQ_BF16>(a, st);                                   \
                 if (e7 != cudaErrorNotSupported) return e7;                                               \
                 cudaError_t e6 = launch_qjl6<RQ_D, PW, RQ_BF16>(a, st);                                   \

@@ -281,6 +281,8 @@ QJL_CASES = [
     (256, 4, 72, L.RQ_CODES_PACKED, torch.float16, 1),
     (256, 3, 128, L.RQ_CODES_INT8, torch.bfloat16, 0),
     (512, 2, 512, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (512, 3, 72, L.RQ_CODES_PACKED, torch.float16, 0),
+    (512, 4, 264, L.RQ_CODES_PACKED, torch.bfloat16, 1),
 ]
 
 
