@@ -173,9 +173,7 @@ template <int PW, bool TWO>
 static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
 {
     if (a.nq > 128) return cudaErrorNotSupported;
-    const size_t smem = sc3_smem(a.nq, a.d, a.m, TWO, PW);
-    if (smem > kMaxSmemPerBlock && sc4_smem(a.nq, a.d, a.m, TWO, PW, 2, 2, 2) > kMaxSmemPerBlock)
-        return cudaErrorNotSupported;
+    if (sc4_smem(a.nq, a.d, a.m, TWO, PW, 2, 2, 2) > kMaxSmemPerBlock) return cudaErrorNotSupported;
     uint16_t *wsB = reinterpret_cast<uint16_t *>(a.workspace);
     const size_t rows = (size_t)a.G * a.nq;
     float *wsN = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.workspace) +
@@ -206,13 +204,7 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
             return cudaGetLastError();
         }
     }
-    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;    // not reached: v4's smallest fits whenever v3 does
-    auto kern = score_v3_kernel<PW, TWO>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(grid > 0 ? grid : 1), kSc3Threads, smem, st>>>(wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms,
-                                                                     a.T, a.G, a.codes, a.norms, *a.tables, a.scores);
-    return cudaGetLastError();
+    return cudaErrorNotSupported;
 }
 
 template <int PW, bool TWO>

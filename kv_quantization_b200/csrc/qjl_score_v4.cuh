@@ -1,7 +1,9 @@
-// qjl_score_v4.cuh -- tensor-core score kernel with eight producer warps (sm_100a).
+// qjl_score_v4.cuh -- warp-specialised tensor-core score kernel (sm_100a).
 //
-// score_v3_kernel (qjl_score_v3.cuh) with the A-operand production split over
-// two sets of four producer warps: set s stages only the packed bytes of the
+// Arithmetic as described in qjl_score_v2.cuh (A = unpacked keys in fp16,
+// B = prologue queries in fp16, two fp32 TMEM accumulators), organised as a
+// producer / MMA / epilogue pipeline that meets only at mbarriers, with the
+// A-operand production split over two sets of four producer warps: set s stages only the packed bytes of the
 // 64-column regions g with g % 2 == s (its own cp.async group, so no thread
 // waits for another's copies) and writes only those regions of each chunk; a
 // chunk is full after eight warp arrivals.  Measured on the pure-QJL KV-cache
@@ -10,9 +12,40 @@
 // allows.  Warps: 0-7 producers, 8 MMA issuer, 9-12 epilogue (TMEM lane
 // quarter = warp mod 4).
 #pragma once
-#include "qjl_score_v3.cuh"
+#include "qjl_score_v2.cuh"
 
 namespace rq {
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Per-thread record row: codes then signs; the row length is an odd number
+// of 8-byte words so that 64-bit reads of 16 consecutive rows hit 32 distinct
+// banks.
+__host__ __device__ inline int sc3_row_bytes(int d, int m, bool two, int pw)
+{
+    const int raw = (two ? d * pw / 8 : 0) + ((m / 8 + 7) & ~7);
+    int w8 = (raw + 7) / 8;
+    if ((w8 & 1) == 0) ++w8;
+    return 8 * w8;
+}
 
 constexpr int kSc4Threads = 13 * 32;
 constexpr int kSc4MaxRing = 4;

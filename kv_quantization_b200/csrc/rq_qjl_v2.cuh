@@ -1,16 +1,12 @@
-// rq_qjl_v2.cuh -- pipelined QJL sketch kernels for d = 128 (sm_100a).
+// rq_qjl_v2.cuh -- pipelined QJL key sketch for d = 128 (sm_100a), and the
+// tcgen05 helpers the later sketch kernels share (TMEM column counts, the
+// MMA issue loop, the sign-word packing).
 //
-// MODE 0 (rq_quantize_qjl): 256 threads quantize a 128-block tile exactly as
-//   quantize_v2_kernel (TMA input ring, 64 values per thread), rebuild the
-//   fp32 reconstruction, form the residual r = x - x^32 and write bf16(r) into
-//   a double-buffered 128 x 128 A tile (128-byte swizzled, K-major); one
-//   thread issues the tcgen05 MMAs of tile i into TMEM accumulator i mod 2
-//   while the threads already work on tile i+1; the sign-packing epilogue of
-//   tile i runs when tile i+2 needs its A buffer back.
-// MODE 1 (qjl_sketch): 3-D TMA loads put 128 keys straight into the A layout
-//   (one 64-column region per load); the threads only compute the canonical
-//   fp32 norms from shared memory; MMA of tile i overlaps the norm pass of
-//   tile i+1 and the epilogue of tile i-1.
+// qjl_v2_sketch_kernel (qjl_sketch; the fallback of rq_sketch_v3.cuh): 3-D
+// TMA loads put 128 keys straight into the A layout (one 64-column region per
+// load); the threads only compute the canonical fp32 norms from shared
+// memory; MMA of tile i overlaps the norm pass of tile i+1 and the epilogue
+// of tile i-1.
 //
 // Epilogue: 8 warps; warp w reads TMEM lanes 32 (w mod 4) .. +31 (its 32
 // vectors) and every other 32-column chunk starting at chunk w / 4, packs the
@@ -120,199 +116,8 @@ __device__ __forceinline__ void stage_projection(const uint16_t *__restrict__ pr
     }
 }
 
-// -------------------------------------------------------------- MODE 0
 
-template <int PW, bool BF16, int STAGES>
-__global__ void __launch_bounds__(kT2, 1)
-qjl_v2_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, const __grid_constant__ QuantTables T,
-                    uint8_t *__restrict__ codes, uint16_t *__restrict__ norms, int m,
-                    const uint16_t *__restrict__ proj, uint8_t *__restrict__ qsigns, uint16_t *__restrict__ qnorms)
-{
-    constexpr int D = 128, TPB = 2;
-    constexpr int CB = kE2 * PW / 8;
-    constexpr int NW = kE2 * PW / 32;
-    const int m16 = qjl_mma_m16(m);
-    const uint32_t ncols = qjl_v2_tmem_cols(m);
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *s_S = base;
-    uint8_t *ring = s_S + (size_t)m16 * 256;
-    uint8_t *s_A = ring + (size_t)STAGES * kTileBytes2;             // 2 x 32 KB
-    uint8_t *lutb = s_A + 2 * 32768;
-    float *bnd = reinterpret_cast<float *>(lutb);
-    float *cent = reinterpret_cast<float *>(lutb + lut_bytes_v2(T));
-    uint32_t *pmask = reinterpret_cast<uint32_t *>(cent + (1 << PW) * 32);
-    uint64_t *full = reinterpret_cast<uint64_t *>(pmask + 64);
-    uint64_t *mma_bar = full + STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 2);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, part = tid & 1;
-    const int64_t nrows = nblocks * TPB;
-    const int64_t ntiles = (nrows + kT2 - 1) / kT2;
-    if (tid == 0) {
-        prefetch_tmap(&tmx);
-        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
-        mbar_init(&mma_bar[0], 1);
-        mbar_init(&mma_bar[1], 1);
-        fence_barrier_init();
-        for (int s = 0; s < STAGES; ++s) {
-            const int64_t t = blockIdx.x + (int64_t)s * gridDim.x;
-            if (t < ntiles) {
-                mbar_arrive_expect_tx(&full[s], kTileBytes2);
-                tma_load_2d(ring + s * kTileBytes2, &tmx, 0, (int)(t * kT2), &full[s]);
-            }
-        }
-    }
-    stage_projection<true>(proj, s_S, m, m16);
-    setup_lut_v2(T, reinterpret_cast<uint2 *>(lutb), bnd);
-    for (int i = tid; i < (1 << PW) * 32; i += kT2) {
-        const int k = i >> 5;
-        cent[i] = k < T.levels ? T.centroid[k] : 0.0f;
-    }
-    setup_pair_masks(T, pmask, D);
-    if (warp == 0) tmem_alloc(tmem_slot, ncols);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t sS = smem_u32(s_S), sA0 = smem_u32(s_A);
-
-    const float2 la = make_float2(T.lut_a, T.lut_a), lb = make_float2(T.lut_b, T.lut_b);
-    const int cells = T.lut_cells, levels = T.levels;
-    const uint32_t cells_m1 = (uint32_t)(cells > 0 ? cells - 1 : 0);
-    const uint8_t *lut_lane = lutb + (lane & 15) * 8;
-    const float *cent_lane = cent + lane;
-    const uint4 *pmv = reinterpret_cast<const uint4 *>(pmask + part * 32);
-    bool ok = true;
-    uint32_t mma_phase[2] = {0u, 0u};
-    int64_t i = 0;
-
-    for (;; ++i) {
-        const int64_t t = blockIdx.x + i * gridDim.x;
-        if (t >= ntiles) break;
-        const int s = (int)(i % STAGES);
-        const bool got = mbar_wait(&full[s], (uint32_t)((i / STAGES) & 1));
-        if (__syncthreads_or(!got)) { ok = false; break; }
-        uint8_t *tile = ring + s * kTileBytes2;
-        uint32_t u[32];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const uint4 v = *sw_row_chunk(tile, tid, k);
-            const uint4 q = pmv[k];
-            u[4 * k] = v.x ^ q.x; u[4 * k + 1] = v.y ^ q.y; u[4 * k + 2] = v.z ^ q.z; u[4 * k + 3] = v.w ^ q.w;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            const int64_t tn = t + (int64_t)STAGES * gridDim.x;
-            if (tn < ntiles) {
-                mbar_arrive_expect_tx(&full[s], kTileBytes2);
-                tma_load_2d(tile, &tmx, 0, (int)(tn * kT2), &full[s]);
-            }
-        }
-        const int64_t row = t * kT2 + tid;
-        const bool valid = row < nrows;
-
-        // ---- quantize (canonical; as quantize_v2_kernel)
-        float2 P[32];
-        row_to_pairs<BF16>(u, P);
-        const float n32 = __fsqrt_rn(combine_parts<TPB>(row_sumsq(P)));
-        fwht_row<TPB>(P, part);
-        const float inv = n32 > 0.0f ? __frcp_rn(n32) : 0.0f;
-        const float2 inv2 = make_float2(inv, inv);
-        uint32_t w[NW];
-#pragma unroll
-        for (int k = 0; k < NW; ++k) w[k] = 0u;
-#pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) {
-            const float2 y = __fmul2_rn(P[i2], inv2);
-            uint32_t c0, c1;
-            if (cells > 0) {
-                const float2 f = __ffma2_rn(y, la, lb);
-                c0 = lut_code_v2(y.x, f.x, lut_lane, cells_m1);
-                c1 = lut_code_v2(y.y, f.y, lut_lane, cells_m1);
-            } else {
-                c0 = bsearch_code(y.x, bnd, levels);
-                c1 = bsearch_code(y.y, bnd, levels);
-            }
-            const int b0 = i2 * PW, b1 = (i2 + 32) * PW;
-            w[b0 >> 5] |= c0 << (b0 & 31);
-            if ((b0 & 31) + PW > 32) w[(b0 >> 5) + 1] |= c0 >> (32 - (b0 & 31));
-            w[b1 >> 5] |= c1 << (b1 & 31);
-            if ((b1 & 31) + PW > 32) w[(b1 >> 5) + 1] |= c1 >> (32 - (b1 & 31));
-        }
-        const uint16_t n16 = norm_to_h16(n32);
-        if (valid) {
-            store_bytes<CB>(codes + row * CB, w);
-            if (part == 0) norms[row / TPB] = n16;
-        }
-
-        // ---- residual r' = s*x - w*scale (fp32, canonical), r = s * r'
-#pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) {
-            P[i2].x = cent_lane[unpack_code<kE2, PW>(w, i2) * 32];
-            P[i2].y = cent_lane[unpack_code<kE2, PW>(w, i2 + 32) * 32];
-        }
-        fwht_row<TPB>(P, part);
-        const float nsc = -__fmul_rn(h16_to_f32(n16), 1.0f / (float)D);
-        const float2 nsc2 = make_float2(nsc, nsc);
-        float2 X[32];
-        row_to_pairs<BF16>(u, X);
-#pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) P[i2] = __fadd2_rn(X[i2], __fmul2_rn(P[i2], nsc2));
-        const float rn32 = __fsqrt_rn(combine_parts<TPB>(row_sumsq(P)));
-        if (valid && part == 0) qnorms[row / TPB] = norm_to_h16(rn32);
-
-        // ---- A buffer a = i mod 2: tile i-2's MMA must be done; drain its accumulator
-        const int a = (int)(i & 1);
-        if (i >= 2) {
-            if (ok && !mbar_wait(&mma_bar[a], mma_phase[a])) ok = false;
-            mma_phase[a] ^= 1u;
-            tc_fence_after();
-            qjl_v2_epilogue(tmem, (uint32_t)(a * m16), m, m16, (t - 2 * (int64_t)gridDim.x) * 128, nblocks, qsigns, ok);
-            tc_fence_before();
-        }
-        uint8_t *A = s_A + a * 32768;
-        const int arow = tid >> 1;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            uint32_t o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int wd = 4 * k + q;
-                const float va = wd < 16 ? P[2 * wd].x : P[2 * wd - 32].y;
-                const float vb = wd < 16 ? P[2 * wd + 1].x : P[2 * wd - 31].y;
-                o[q] = pack2<true>(va, vb);
-            }
-            const uint4 q = pmv[k];
-            *reinterpret_cast<uint4 *>(A + part * 16384 + sw128_offset(arow, k)) =
-                make_uint4(o[0] ^ q.x, o[1] ^ q.y, o[2] ^ q.z, o[3] ^ q.w);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        if (tid == 0) {
-            tc_fence_after();
-            qjl_v2_issue(sA0 + (uint32_t)a * 32768u, sS, m16, tmem + (uint32_t)(a * m16));
-            mma_commit(&mma_bar[a]);
-        }
-    }
-    // drain the last two tiles (i = number of tiles this CTA processed)
-    for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j) {
-        const int a = (int)(j & 1);
-        if (ok && !mbar_wait(&mma_bar[a], mma_phase[a])) ok = false;
-        mma_phase[a] ^= 1u;
-        tc_fence_after();
-        qjl_v2_epilogue(tmem, (uint32_t)(a * m16), m, m16, (blockIdx.x + j * (int64_t)gridDim.x) * 128, nblocks, qsigns,
-                        ok);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, ncols);
-}
-
-// -------------------------------------------------------------- MODE 1
+// -------------------------------------------------------------- key sketch
 
 // 3-D view of the keys: {64 values, 2 chunks, n tokens}; box {64, 1, 128}.
 template <bool BF16, int STAGES>
