@@ -426,9 +426,9 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
     if (!rq::make_rows64_tmap(&a.tmap_x, x, n / 64)) return RQ_ECUDA;
     a.has_tmap_v = qjl && rq::make_vectors_tmap(&a.tmap_v, x, n / d, d);
     a.has_tmap_v32 = !qjl && d == 128 && rq::make_vectors_tmap(&a.tmap_v32, x, n / d, d, 32);
-    if (qjl && d == 512) {
+    if (qjl && d >= 128) {
         const int m16 = (m + 15) / 16 * 16;
-        a.has_tmap_s = rq::make_proj_tmap(&a.tmap_s, proj, m, d, m16 < 256 ? m16 : 256);
+        a.has_tmap_s = (m16 <= 256 || m16 % 256 == 0) && rq::make_proj_tmap(&a.tmap_s, proj, m, d, m16 < 256 ? m16 : 256);
     }
     return cuda_status(rq::launch_quantize(a, stream));
 }

@@ -264,7 +264,7 @@ static cudaError_t launch_qjl7(const QuantArgs &a, cudaStream_t st)
     if constexpr (D != 256) {
         return cudaErrorNotSupported;
     } else {
-        if (!a.has_tmap_v || a.tables->sat_cells <= 0) return cudaErrorNotSupported;
+        if (!a.has_tmap_v || !a.has_tmap_s || a.tables->sat_cells <= 0) return cudaErrorNotSupported;
         if ((size_t)qjl_v7_nacc(a.m) * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
         const size_t smem = qjl_v7_smem(a.m, *a.tables);
         if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
@@ -277,7 +277,7 @@ static cudaError_t launch_qjl7(const QuantArgs &a, cudaStream_t st)
         const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
         kern<<<(unsigned)(grid > 0 ? grid : 1), kW7 * 32, smem, st>>>(
             a.tmap_v, a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms, a.m,
-            static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
+            a.tmap_s, a.qsigns, a.qnorms);
         return cudaGetLastError();
     }
 }
@@ -288,7 +288,7 @@ static cudaError_t launch_qjl6(const QuantArgs &a, cudaStream_t st)
     if constexpr (D != 128) {
         return cudaErrorNotSupported;
     } else {
-        if (!a.has_tmap_v || a.tables->sat_cells <= 0) return cudaErrorNotSupported;
+        if (!a.has_tmap_v || !a.has_tmap_s || a.tables->sat_cells <= 0) return cudaErrorNotSupported;
         if ((size_t)kGroups6 * qjl_v6_nacc(a.m) * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
         const size_t smem = qjl_v6_smem(a.m, *a.tables);
         if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
@@ -302,7 +302,7 @@ static cudaError_t launch_qjl6(const QuantArgs &a, cudaStream_t st)
         const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
         kern<<<(unsigned)(grid > 0 ? grid : 1), kW6 * 32, smem, st>>>(
             a.tmap_v, a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms, a.m,
-            static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
+            a.tmap_s, a.qsigns, a.qnorms);
         return cudaGetLastError();
     }
 }

@@ -31,29 +31,32 @@ constexpr int kGroups6 = 2;                   // groups of eight warps
 constexpr int kNSG6 = 2;                      // tile ring depth per group
 constexpr uint32_t kTileBytes6 = 128u * 256u;  // 128 blocks x 2 regions x 128 B
 
-// Stage S' = S diag(s) (the sign diagonal folded into the projection's
+// S (m16 rows x D columns, 16-bit) into the tcgen05 B layout by 2-D TMA, one
+// box of min(m16, 256) rows per 64-column region (rows >= m are zero-filled);
+// issued by one thread, completion counted on `bar`.
+template <int D>
+__device__ __forceinline__ void tma_stage_projection(const CUtensorMap *tms, uint8_t *s_S, int m16, uint64_t *bar)
+{
+    mbar_arrive_expect_tx(bar, (uint32_t)m16 * 128u * (uint32_t)(D / 64));
+    for (int kc = 0; kc < D / 64; ++kc)
+        for (int r0 = 0; r0 < m16; r0 += 256)
+            tma_load_2d(s_S + (size_t)kc * m16 * 128 + (size_t)r0 * 128, tms, 64 * kc, r0, bar);
+}
+
+// S' = S diag(s) in place (the sign diagonal folded into the projection's
 // columns: a bf16 sign flip is exact, so P = r' S'^T = r S^T bit for bit with
-// r' = s * r the residual before its final sign flip) in the tcgen05 B layout.
-template <int D, bool SIGNS>
-__device__ __forceinline__ void stage_projection_signed(const uint16_t *__restrict__ proj, uint8_t *s_S, int m,
-                                                        int m16, const QuantTables &T)
+// r' = s * r the residual before its final sign flip): every 16-byte chunk
+// (8 columns of one row) XORed with the pair masks of its columns.
+template <int D>
+__device__ __forceinline__ void sign_fold_projection(uint8_t *s_S, int m16, const uint32_t *pmask)
 {
     for (int idx = threadIdx.x; idx < m16 * (D / 8); idx += blockDim.x) {
         const int i = idx / (D / 8), c = idx % (D / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (i < m) v = __ldg(reinterpret_cast<const uint4 *>(proj + (size_t)i * D) + c);
-        if constexpr (SIGNS) {
-            uint32_t x[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = 8 * c + 2 * e;            // values j, j + 1 of the row
-                const uint32_t b0 = (T.sign_words[j >> 5] >> (j & 31)) & 1u;
-                const uint32_t b1 = (T.sign_words[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u;
-                x[e] ^= (b0 << 15) | (b1 << 31);
-            }
-            v = make_uint4(x[0], x[1], x[2], x[3]);
-        }
-        *reinterpret_cast<uint4 *>(s_S + (size_t)(c >> 3) * m16 * 128 + sw128_offset(i, c & 7)) = v;
+        uint4 *p = reinterpret_cast<uint4 *>(s_S + (size_t)(c >> 3) * m16 * 128 + sw128_offset(i, c & 7));
+        const uint4 q = *reinterpret_cast<const uint4 *>(pmask + 4 * c);
+        uint4 v = *p;
+        v.x ^= q.x; v.y ^= q.y; v.z ^= q.z; v.w ^= q.w;
+        *p = v;
     }
 }
 
@@ -228,14 +231,14 @@ __host__ __device__ inline uint32_t qjl_v6_tmem_cols(int m)
 __host__ __device__ inline size_t qjl_v6_smem(int m, const QuantTables &T)
 {
     return 1024 + (size_t)qjl_mma_m16(m) * 256 + (size_t)kGroups6 * kNSG6 * kTileBytes6 +
-           (size_t)T.sat_cells * 128 + 256 + 8 * (kGroups6 * (2 * kNSG6 + 2)) + 16 + 8 * kGroups6;
+           (size_t)T.sat_cells * 128 + 256 + 8 * (kGroups6 * (2 * kNSG6 + 2) + 1) + 16 + 8 * kGroups6;
 }
 
 template <int PW, bool BF16, bool SIGNS>
 __global__ void __launch_bounds__(kW6 * 32, 1)
 qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, const __grid_constant__ QuantTables T,
                     uint8_t *__restrict__ codes, uint16_t *__restrict__ norms, int m,
-                    const uint16_t *__restrict__ proj, uint8_t *__restrict__ qsigns, uint16_t *__restrict__ qnorms)
+                    const __grid_constant__ CUtensorMap tms, uint8_t *__restrict__ qsigns, uint16_t *__restrict__ qnorms)
 {
     constexpr int CB = 16 * PW;                     // code bytes per block
     constexpr int HB = 8 * PW;                      // code bytes per half block
@@ -251,7 +254,8 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
     uint64_t *full = reinterpret_cast<uint64_t *>(pmask + 64);
     uint64_t *mma_done = full + kGroups6 * kNSG6;
     uint64_t *acc_full = mma_done + kGroups6 * kNSG6;
-    uint32_t *ready = reinterpret_cast<uint32_t *>(acc_full + kGroups6 * 2);
+    uint64_t *s_ready = acc_full + kGroups6 * 2;
+    uint32_t *ready = reinterpret_cast<uint32_t *>(s_ready + 1);
     uint32_t *tmem_slot = ready + kGroups6;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -275,17 +279,24 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
             mbar_init(&mma_done[i], 1);
         }
         for (int i = 0; i < kGroups6 * 2; ++i) mbar_init(&acc_full[i], 1);
+        mbar_init(s_ready, 1);
         for (int i = 0; i < kGroups6; ++i) ready[i] = 0u;
         fence_barrier_init();
     }
     __syncthreads();
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tms);
+        tma_stage_projection<128>(&tms, s_S, m16, s_ready);
+    }
     if (lw == 0 && lane == 0)
         for (int k = 0; k < kNSG6; ++k)
             if (tile_of(k) < t1) load_tile(k);
-    stage_projection_signed<128, SIGNS>(proj, s_S, m, m16, T);
     setup_sat_lut16(T, reinterpret_cast<uint4 *>(lutb));
     setup_pair_masks(T, pmask, 128);
     if (warp == 0) tmem_alloc(tmem_slot, ncols);
+    __syncthreads();                                // masks written
+    bool ok = mbar_wait(s_ready, 0u);               // S landed
+    if (SIGNS) sign_fold_projection<128>(s_S, m16, pmask);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -296,7 +307,6 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
     const uint32_t pmh = smem_u32(pmask) + (uint32_t)hf * 128u;
     const uint32_t sS = smem_u32(s_S);
     const int eq = lw & 3, ech = lw >> 2;           // epilogue: TMEM lane quarter, column-chunk parity
-    bool ok = true;
 
     auto epilogue = [&](int64_t kk) {
         const int a = nacc == 2 ? (int)(kk & 1) : 0;

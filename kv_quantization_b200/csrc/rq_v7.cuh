@@ -33,14 +33,14 @@ __host__ __device__ inline uint32_t qjl_v7_tmem_cols(int m)
 
 __host__ __device__ inline size_t qjl_v7_smem(int m, const QuantTables &T)
 {
-    return 1024 + (size_t)qjl_mma_m16(m) * 512 + kTileBytes7 + (size_t)T.sat_cells * 128 + 512 + 8 * 4 + 16;
+    return 1024 + (size_t)qjl_mma_m16(m) * 512 + kTileBytes7 + (size_t)T.sat_cells * 128 + 512 + 8 * 5 + 16;
 }
 
 template <int PW, bool BF16, bool SIGNS>
 __global__ void __launch_bounds__(kW7 * 32, 1)
 qjl_v7_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, const __grid_constant__ QuantTables T,
                     uint8_t *__restrict__ codes, uint16_t *__restrict__ norms, int m,
-                    const uint16_t *__restrict__ proj, uint8_t *__restrict__ qsigns, uint16_t *__restrict__ qnorms)
+                    const __grid_constant__ CUtensorMap tms, uint8_t *__restrict__ qsigns, uint16_t *__restrict__ qnorms)
 {
     constexpr int CB = 32 * PW;                     // code bytes per block
     constexpr int QB = 8 * PW;                      // code bytes per 64-value part
@@ -56,7 +56,8 @@ qjl_v7_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
     uint64_t *full = reinterpret_cast<uint64_t *>(pmask + 128);
     uint64_t *mma_done = full + 1;
     uint64_t *acc_full = mma_done + 1;                              // [2]
-    uint32_t *ready = reinterpret_cast<uint32_t *>(acc_full + 2);
+    uint64_t *s_ready = acc_full + 2;
+    uint32_t *ready = reinterpret_cast<uint32_t *>(s_ready + 1);
     uint32_t *tmem_slot = ready + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -74,15 +75,22 @@ qjl_v7_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
         mbar_init(mma_done, 1);
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
+        mbar_init(s_ready, 1);
         *ready = 0u;
         fence_barrier_init();
     }
     __syncthreads();
-    if (threadIdx.x == 0 && t0 < t1) load_tile(t0);
-    stage_projection_signed<256, SIGNS>(proj, s_S, m, m16, T);
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tms);
+        tma_stage_projection<256>(&tms, s_S, m16, s_ready);
+        if (t0 < t1) load_tile(t0);
+    }
     setup_sat_lut16(T, reinterpret_cast<uint4 *>(lutb));
     setup_pair_masks(T, pmask, 256);
     if (warp == 0) tmem_alloc(tmem_slot, ncols);
+    __syncthreads();                                // masks written
+    bool ok = mbar_wait(s_ready, 0u);               // S landed
+    if (SIGNS) sign_fold_projection<256>(s_S, m16, pmask);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -95,7 +103,6 @@ qjl_v7_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
     const uint32_t tile = smem_u32(tile_b);
     const uint32_t rbase = tile + (uint32_t)q * 16384u;
     const int eq = warp & 3, ech = warp >> 2;       // epilogue: TMEM lane quarter, first 32-column chunk
-    bool ok = true;
 
     auto epilogue = [&](int64_t kk) {
         const int a = nacc == 2 ? (int)(kk & 1) : 0;
