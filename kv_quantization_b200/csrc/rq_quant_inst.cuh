@@ -218,10 +218,24 @@ static cudaError_t launch_dq5(const DequantArgs &a, cudaStream_t st)
         return cudaErrorNotSupported;
     } else {
         if (!a.has_tmap_out32) return cudaErrorNotSupported;
-        const size_t smem = dequantize_v5_smem(PW, a.tables->levels);
-        if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
         const bool signs = a.tables->sign_words[0] | a.tables->sign_words[1] | a.tables->sign_words[2] |
                            a.tables->sign_words[3];
+        if constexpr (PW <= 3) {                    // pair layout (rq_v5.cuh): measured faster up to 3 bits only
+            const size_t smemp = dequantize_v5p_smem(PW);
+            if (smemp <= kMaxSmemPerBlock && a.tables->levels == (1 << PW)) {
+                auto kp = signs ? dequantize_v5p_kernel<PW, BF16, true> : dequantize_v5p_kernel<PW, BF16, false>;
+                cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemp);
+                if (e != cudaSuccess) return e;
+                const int64_t chunks = (a.nblocks + 31) / 32;
+                const int64_t want = (chunks + kW5 - 1) / kW5;
+                const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
+                kp<<<(unsigned)(grid > 0 ? grid : 1), kW5 * 32, smemp, st>>>(
+                    static_cast<const uint8_t *>(a.codes), a.norms, a.nblocks, *a.tables, a.tmap_out32);
+                return cudaGetLastError();
+            }
+        }
+        const size_t smem = dequantize_v5_smem(PW, a.tables->levels);
+        if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
         auto kern = signs ? dequantize_v5_kernel<PW, BF16, true> : dequantize_v5_kernel<PW, BF16, false>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

@@ -436,4 +436,162 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
     if (lane == 0) bulk_wait<0>();
 }
 
+// ------------------------------------------------------------------ dequantize, pair layout
+//
+// For codes of up to 3 bits (where it measured faster: the 4- and 5-bit pair
+// tables are 32 KB and lose more to latency and bank conflicts than the halved
+// lookups save) the block is held as 64 float2 Q[i] = (v_2i, v_2i+1):
+// the 2*PW-bit field of a value pair indexes a table of centroid pairs (one
+// 8-byte load and one field extraction per two values), the Hadamard stage
+// h = 1 is the add/sub inside each float2 and h = 2..64 are packed operations
+// on the pair index, and the bf16/fp16 output words are the pairs themselves.
+// The arithmetic (stage order, roundings) is the canonical one, as above.
+
+__host__ __device__ inline int pair_copies5(int pw) { return pw <= 3 ? 16 : (pw == 4 ? 16 : 4); }
+
+__host__ __device__ inline size_t dequantize_v5p_smem(int pw)
+{
+    return 1024 + (size_t)kW5 * kChunkBytes5 + (size_t)kW5 * kNSD5 * 512 * pw +
+           ((size_t)1 << (2 * pw)) * pair_copies5(pw) * 8 + 256 + 8 * kW5 * kNSD5;
+}
+
+__device__ __forceinline__ void fwht128_pairs(float2 *Q)
+{
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {                      // stage h = 1
+        const float a = Q[i].x, b = Q[i].y;
+        Q[i].x = __fadd_rn(a, b);
+        Q[i].y = __fsub_rn(a, b);
+    }
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int h = 1; h < 64; h *= 2) {                   // stages 2h = 2 .. 64 on the pair index
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            if (i & h) continue;
+            const float2 a = Q[i], b = Q[i + h];
+            Q[i] = __fadd2_rn(a, b);
+            Q[i + h] = __ffma2_rn(b, m1, a);
+        }
+    }
+}
+
+template <bool OUT_BF16, bool SIGNS>
+__device__ __forceinline__ void store_row128_pairs(uint32_t tile, uint32_t half_bytes, int r, uint32_t pmask_smem,
+                                                   const float2 *Q)
+{
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {                      // 16-byte chunk k = values 8k .. 8k+7
+        uint4 v;
+        v.x = pack2<OUT_BF16>(Q[4 * k + 0].x, Q[4 * k + 0].y);
+        v.y = pack2<OUT_BF16>(Q[4 * k + 1].x, Q[4 * k + 1].y);
+        v.z = pack2<OUT_BF16>(Q[4 * k + 2].x, Q[4 * k + 2].y);
+        v.w = pack2<OUT_BF16>(Q[4 * k + 3].x, Q[4 * k + 3].y);
+        if constexpr (SIGNS) {
+            const uint4 mk = lds128_fresh(pmask_smem + 16u * k);
+            v.x ^= mk.x; v.y ^= mk.y; v.z ^= mk.z; v.w ^= mk.w;
+        }
+        sts128(tile + (uint32_t)(k >> 3) * half_bytes + sw128_offset(r, k & 7), v);
+    }
+}
+
+template <int PW, bool BF16, bool SIGNS>
+__global__ void __launch_bounds__(kW5 * 32, 1)
+dequantize_v5p_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ norms, int64_t nblocks,
+                      const __grid_constant__ QuantTables T, const __grid_constant__ CUtensorMap tmo)
+{
+    static_assert(PW <= 5, "pair table of 2^(2 PW) entries");
+    constexpr int CB = 16 * PW;
+    constexpr uint32_t RING = 512u * PW;
+    constexpr int NE = 1 << (2 * PW);               // centroid pairs
+    constexpr int CP = PW <= 4 ? 16 : 4;            // copies (lane % CP reads its own)
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *outb = base;
+    uint8_t *cring = outb + (size_t)kW5 * kChunkBytes5;
+    float2 *ptab = reinterpret_cast<float2 *>(cring + (size_t)kW5 * kNSD5 * RING);
+    uint32_t *pmask = reinterpret_cast<uint32_t *>(ptab + NE * CP);
+    uint64_t *full = reinterpret_cast<uint64_t *>(pmask + 64);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nchunks = (nblocks + 31) / 32;
+    int64_t c0, c1;
+    cta_chunks(nchunks, c0, c1);
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmo);
+        for (int s = 0; s < kW5 * kNSD5; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    for (int i = threadIdx.x; i < NE * CP; i += blockDim.x) {
+        const int e = i / CP;
+        ptab[i] = make_float2(T.centroid[e & ((1 << PW) - 1)], T.centroid[e >> PW]);
+    }
+    setup_pair_masks(T, pmask, 128);
+    __syncthreads();
+
+    uint8_t *wring = cring + (size_t)warp * kNSD5 * RING;
+    uint8_t *wout = outb + (size_t)warp * kChunkBytes5;
+    uint64_t *wfull = full + warp * kNSD5;
+    auto issue = [&](int64_t j, int s) {
+        const int64_t nb = nblocks - j * 32 < 32 ? nblocks - j * 32 : 32;
+        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(nb * CB));
+        bulk_load(wring + (size_t)s * RING, codes + j * 32 * CB, (uint32_t)(nb * CB), &wfull[s]);
+    };
+    if (lane == 0)
+        for (int s = 0; s < kNSD5; ++s) {
+            const int64_t j = c0 + warp + (int64_t)s * kW5;
+            if (j < c1) issue(j, s);
+        }
+    const uint32_t ptab_lane = smem_u32(ptab) + (uint32_t)(lane & (CP - 1)) * 8u;
+    const uint32_t pm = smem_u32(pmask);
+    auto fetch_norm = [&](int64_t j) -> float {
+        const int64_t blk = j * 32 + lane;
+        return (j < c1 && blk < nblocks) ? h16_to_f32(__ldg(norms + blk)) : 0.0f;
+    };
+    float nrm = fetch_norm(c0 + warp);
+
+    for (int64_t k = 0;; ++k) {
+        const int64_t j = c0 + warp + k * kW5;
+        if (j >= c1) break;
+        const int s = (int)(k % kNSD5);
+        const float nrm_next = fetch_norm(j + kW5);
+        if (!mbar_wait(&wfull[s], (uint32_t)((k / kNSD5) & 1))) break;
+        uint32_t cw[4 * PW];
+        const uint32_t src = smem_u32(wring + (size_t)s * RING) + (uint32_t)lane * CB;
+#pragma unroll
+        for (int q = 0; q < PW; ++q) {
+            const uint4 v = lds128(src + 16u * q);
+            cw[4 * q] = v.x; cw[4 * q + 1] = v.y; cw[4 * q + 2] = v.z; cw[4 * q + 3] = v.w;
+        }
+        __syncwarp();
+        if (lane == 0 && j + (int64_t)kNSD5 * kW5 < c1) issue(j + (int64_t)kNSD5 * kW5, s);
+        float2 Q[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const uint32_t e = unpack_code<64, 2 * PW>(cw, i);         // codes of values 2i (low) and 2i+1
+            uint2 v;
+            asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(ptab_lane + e * (uint32_t)(CP * 8)));
+            Q[i] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+        }
+        fwht128_pairs(Q);
+        const float sc = __fmul_rn(nrm, 1.0f / 128.0f);
+        const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) Q[i] = __fmul2_rn(Q[i], sc2);
+        uint8_t *ob = wout;
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        store_row128_pairs<BF16, SIGNS>(smem_u32(ob), kChunkBytes5 / 2, lane, pm, Q);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_3d(&tmo, 0, 0, (int)(j * 32), ob);
+            tma_store_3d(&tmo, 0, 1, (int)(j * 32), ob + kChunkBytes5 / 2);
+            bulk_commit();
+        }
+        nrm = nrm_next;
+    }
+    if (lane == 0) bulk_wait<0>();
+}
+
 }  // namespace rq
