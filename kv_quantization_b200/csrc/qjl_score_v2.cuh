@@ -107,7 +107,8 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
         float acc0 = 0.0f, acc1 = 0.0f;
         if (i < m) {
             const uint4 *Srow = reinterpret_cast<const uint4 *>(proj + (int64_t)i * d);
-            for (int j8 = 0; j8 < d / 8; ++j8) {
+#pragma unroll 4
+            for (int j8 = 0; j8 < d / 8; ++j8) {                 // d / 8 is a multiple of 8
                 const uint4 w = __ldg(Srow + j8);
                 const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
