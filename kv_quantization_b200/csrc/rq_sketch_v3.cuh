@@ -10,8 +10,9 @@
 //            acc_full;
 //   warps 2-5 norms: thread = key, canonical fp32 pairwise norm of its 128
 //            values read from the stage, arrive stage_free;
-//   warps 6-9 epilogue: TMEM lane quarter (warp mod 4) = 32 keys, all column
-//            chunks loaded back to back, sign words stored, arrive acc_free.
+//   warps 6-13 epilogue: TMEM lane quarter (warp mod 4) = 32 keys, half of
+//            the 32-column chunks each (two warps per quarter), loaded two at
+//            a time, sign words stored, arrive acc_free.
 // A stage returns to the TMA warp when both its MMA and its norm pass are done
 // (stage_free counts 4 norm-warp arrivals + 1 MMA commit).
 #pragma once
@@ -19,7 +20,7 @@
 
 namespace rq {
 
-constexpr int kSk3Warps = 10;
+constexpr int kSk3Warps = 14;
 
 __device__ __forceinline__ void mbar_arrive_cta(uint64_t *bar)
 {
@@ -60,7 +61,7 @@ sketch_v3_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_free[a], 4);                     // 4 epilogue warps
+            mbar_init(&acc_free[a], 8);                     // 8 epilogue warps
         }
         mbar_init(&s_ready[0], 1);
         fence_barrier_init();
@@ -139,30 +140,33 @@ sketch_v3_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
+        const int part = (warp - 6) >> 2;                   // which half of the column chunks
+        const int nchk = (m16 + 31) / 32, half = (nchk + 1) / 2;
+        const int ch0 = part * half, ch1 = min(nchk, ch0 + half);
         for (int64_t i = 0; i < my_tiles && ok; ++i) {
             const int a = (int)(i & 1);
             if (!mbar_wait(&acc_full[a], (uint32_t)((i >> 1) & 1))) { ok = false; break; }
             tc_fence_after();
             const int64_t tok = (blockIdx.x + i * gridDim.x) * 128 + quarter * 32 + lane;
             uint8_t *dst = signs + tok * (m / 8);
-            for (int c0 = 0; c0 < m16; c0 += 128) {
-                uint32_t acc[4][32];
-                const int nch = min(4, (m16 - c0 + 31) / 32);
+            for (int ch = ch0; ch < ch1; ch += 2) {
+                uint32_t acc[2][32];
+                const int nch = min(2, ch1 - ch);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int q = 0; q < 2; ++q)
                     if (q < nch)
-                        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * m16 + c0 + 32 * q), acc[q]);
+                        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * m16 + 32 * (ch + q)), acc[q]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int cc = c0 + 32 * q;
+                for (int q = 0; q < 2; ++q) {
+                    const int cc = 32 * (ch + q);
                     if (q < nch && tok < nvec && cc < m) {
                         const uint32_t word = sign_word(acc[q]);
                         const int nb = min(4, (m - cc) / 8);
                         if (nb == 4 && (m & 31) == 0) {
                             *reinterpret_cast<uint32_t *>(dst + cc / 8) = word;
                         } else {
-                            for (int b = 0; b < nb; ++b) dst[cc / 8 + b] = (uint8_t)(word >> (8 * b));
+                            for (int bb = 0; bb < nb; ++bb) dst[cc / 8 + bb] = (uint8_t)(word >> (8 * bb));
                         }
                     }
                 }
