@@ -43,22 +43,24 @@ __host__ __device__ inline size_t qjl_v2_smem(int mode, int pw, int m, const Qua
 
 // Bit i of the result = (v[i] >= 0) for 32 fp32 values.  Adding +0 maps -0
 // to +0 (and leaves every other value unchanged), so the bit is the inverted
-// sign bit; the 32 shifts are independent and combine in an OR tree.
+// sign bit.  The additions run on pairs; for each g = 0..7 two byte permutes
+// gather the top bytes of v[g], v[g+8], v[g+16], v[g+24] into bytes 0..3 of
+// one word, whose bit 7 of byte b is then the sign of v[8b+g], moved to bit
+// 8b+g with one shift and one masked OR.
 __device__ __forceinline__ uint32_t sign_word(const uint32_t *v)
 {
-    uint32_t part[8];
+    const float2 z = make_float2(0.0f, 0.0f);
+    uint32_t neg = 0u;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
-        uint32_t b[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = 4 * g + k;
-            const uint32_t x = __float_as_uint(__fadd_rn(__uint_as_float(v[i]), 0.0f));
-            b[k] = (x >> 31) << i;                       // 1 where negative
-        }
-        part[g] = (b[0] | b[1]) | (b[2] | b[3]);
+        const float2 lo = __fadd2_rn(make_float2(__uint_as_float(v[g]), __uint_as_float(v[g + 8])), z);
+        const float2 hi = __fadd2_rn(make_float2(__uint_as_float(v[g + 16]), __uint_as_float(v[g + 24])), z);
+        const uint32_t top = __byte_perm(__byte_perm(__float_as_uint(lo.x), __float_as_uint(lo.y), 0x0073u),
+                                         __byte_perm(__float_as_uint(hi.x), __float_as_uint(hi.y), 0x0073u),
+                                         0x5410u);
+        neg |= (top >> (7 - g)) & (0x01010101u << g);
     }
-    return ~(((part[0] | part[1]) | (part[2] | part[3])) | ((part[4] | part[5]) | (part[6] | part[7])));
+    return ~neg;
 }
 
 // Sign-pack epilogue of one 128-vector tile from TMEM accumulator columns
