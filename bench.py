@@ -150,7 +150,7 @@ def job_rate(units_per_rank_step, world, steps, max_ms):
 # DRAM bytes (read + write) of one 4-bit launch of each headline kernel, measured with
 # ncu (--set full) on the 8192 x 8192 weight; scaled to a workload by element count.
 # Writes still dirty in L2 when a kernel ends are not in the DRAM count.
-NCU_DRAM_BYTES_8192SQ = {"qjl_v6": 134.53e6 + 24.63e6, "dequantize_v5": 34.65e6 + 75.14e6}
+NCU_DRAM_BYTES_8192SQ = {"qjl_v6": 134.53e6 + 25.83e6, "dequantize_v5": 34.65e6 + 74.65e6}
 
 
 def alg_bytes_quant(n, bits):
