@@ -339,6 +339,29 @@ def test_score_pure_qjl():
     assert np.all(err <= _score_tol(q16, G, nq, d, kn.cpu().numpy().view(np.uint16)))
 
 
+def test_score_fp16_projection_ragged_queries():
+    """Pure QJL score with the projection given in fp16 (the same matrix as the
+    bf16 one the keys were sketched with, widened exactly) and 33 queries, so
+    the query projection reads fp16 S and the second 32-query group is ragged."""
+    G, nq, T, d, m = 2, 33, 200, 128, 128
+    k = synth.kv_with_channels(1, G, T, d, seed=21, device=DEV).reshape(-1)
+    q = synth.normal((G, nq, d), seed=22, device=DEV)
+    S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
+    L.qjl_make_projection(12, m, d, S)
+    signs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=DEV)
+    kn = torch.empty(G * T, dtype=torch.int16, device=DEV)
+    L.qjl_sketch(k, d, m, S, signs, kn)
+    S16 = S.to(torch.float16)
+    scores = torch.empty(G, nq, T, dtype=torch.float32, device=DEV)
+    ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
+    L.qjl_score(q, G, nq, d, m, S16, signs, kn, T, scores, ws)
+    torch.cuda.synchronize()
+    q16 = u16(q)
+    want = O.score(q16, G, nq, d, m, u16(S16), O.F16, signs.cpu().numpy(), kn.cpu().numpy().view(np.uint16), T)
+    err = np.abs(scores.cpu().numpy().astype(np.float64) - want)
+    assert np.all(err <= _score_tol(q16, G, nq, d, kn.cpu().numpy().view(np.uint16)))
+
+
 @pytest.mark.parametrize("d", [256, 512])
 def test_score_two_stage(d):
     """2-bit rotated Lloyd-Max keys + QJL (m = d) residual sketch, 32 queries."""
