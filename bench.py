@@ -1,25 +1,33 @@
 """Benchmark of the rotated-quantization + QJL hot path on B200.
 
-One step = the whole path over one 4096 x 4096 bf16 weight (Student-t nu=4,
-std 0.02, 0.1% outliers x20; d = 128; seeded signs): for bits 3, 4 and 5,
-rq_quantize_qjl (norm, sign flip, Walsh-Hadamard, Lloyd-Max search, packed
-codes, fused residual + 1-bit QJL sketch with m = 128) then rq_dequantize.
-Metric: quantize+dequantize input GB/s = 3 x 33.55 MB / step time, with L2
-flushed between steps (inputs fit in L2).  Secondary: QJL score tokens/s on
-the KV-cache (4 x 8 x 32768 keys, head_dim 128, m = 256, 32 queries) and the
-TurboQuant-style 3-bit keys (131072 x 8, head_dim 256, 2-bit + QJL m = d).
+Headline (one step = the whole path over one batch of input): all linears of
+32 Llama-7B-shaped decoder layers in bf16 (per layer q/k/v/o 4096x4096,
+gate/up 11008x4096, down 4096x11008; 6.48e9 values, 13 GB), entries
+N(0, 0.02^2) times a per-output-row scale exp(U[ln 1/2, ln 2]); d = 128,
+4-bit Lloyd-Max codes packed, sign diagonal seeded 1000 + layer.  Per layer one
+rq_quantize call (the layer's seven matrices are contiguous) then one
+rq_dequantize call.  Metric: quantize+dequantize input GB/s = 2 bytes x 6.48e9
+/ step time.  The input is 100x the L2, so no flush is needed.
+
+Secondary lines (each its own roofline): the 256x512 fp16 weight round trip
+(latency), the 4096x4096 bf16 weight with outliers at 3/4/5 bits with the
+fused QJL residual sketch (m = 128), the KV cache 4x8x32768x128 (V: 4-bit
+round trip; K: QJL m = 256 sketch and the pure-QJL score of 32 queries per
+head), and TurboQuant-style 3-bit keys (2-bit + QJL m = d) at head dim 256
+and 512 for 131072 tokens x 8 heads, with their scores.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-N > 1 runs one replica per GPU (torchrun; nothing is exchanged but the
-barrier and the max-over-ranks step time).
+--gpus N > 1 runs one independent replica per GPU (relaunching itself under
+torch.distributed.run when started without it); nothing is exchanged but a
+barrier and the max-over-ranks step time.
 """
 from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -31,25 +39,29 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-D, M = 128, 128
-BITS = (3, 4, 5)
-ROWS = COLS = 4096
-SIGN_SEED, PROJ_SEED = 1, 2
-WORKLOAD = "weight 4096x4096 bf16 student-t(4) std 0.02 + 0.1% outliers x20; d=128; bits 3,4,5 packed; " \
-           "seeded signs; fused QJL residual sketch m=128; quantize+dequantize"
+D, BITS = 128, 4
+LAYERS = 32
+LLAMA7B = ((4096, 4096),) * 4 + ((11008, 4096),) * 2 + ((4096, 11008),)   # q k v o gate up down
+LAYER_N = sum(r * c for r, c in LLAMA7B)                                # 202,375,168
+WORKLOAD = ("all linears of 32 Llama-7B-shaped decoder layers, bf16 (6,476,005,376 values; per layer q/k/v/o "
+            "4096x4096, gate/up 11008x4096, down 4096x11008), N(0,0.02^2) x per-row exp(U[ln .5, ln 2]); "
+            "d=128, 4-bit packed Lloyd-Max, signs seeded 1000+layer; per layer rq_quantize then rq_dequantize")
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="rq", choices=["rq", "reference"])
     p.add_argument("--no-secondary", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
-    p.add_argument("--kernels-once", action="store_true",
-                   help="run each hot kernel once on inputs larger than L2 (profiling driver), print nothing else")
-    return p.parse_args()
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--profile", default=None,
+                   help="run one case's kernels once (profiling driver): c3_layer, weight4096_fused, kv_sketch, "
+                        "kv_score, kv_v, tq256, tq512; print nothing else")
+    p.add_argument("--rank-selftest", action="store_true", help=argparse.SUPPRESS)
+    return p.parse_args(argv)
 
 
 def peaks():
@@ -61,8 +73,26 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def roofline_hbm(alg_bytes, ms, traffic=None, **extra):
+    hbm, _, src = peaks()
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    r = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+         "peak_source": src, "traffic": traffic}
+    r.update(extra)
+    return r
+
+
+def roofline_tensor(flops, ms, **extra):
+    _, tf, src = peaks()
+    t = flops / (ms * 1e-3) / 1e12
+    r = {"bound": "tensor", "achieved": round(t, 2), "peak": tf, "unit": "TFLOP/s", "frac": round(t / tf, 4),
+         "peak_source": src}
+    r.update(extra)
+    return r
+
+
 class Clocks:
-    """nvidia-smi samples (every 20 ms) kept for the timed window only."""
+    """nvidia-smi samples (every 20 ms), kept for the timed window only."""
 
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -122,13 +152,7 @@ class Clocks:
                 "samples": len(sm)}
 
 
-# ---------------------------------------------------------------------------- device arm
-
-def make_inputs(dev):
-    import torch
-    from kv_quantization_b200 import synth
-    return synth.student_t_outliers(ROWS, COLS, seed=1, device=dev).reshape(-1)
-
+# ---------------------------------------------------------------------------- replicas
 
 def reduce_max_ms(total_ms, world, device=None):
     """Max over ranks of the per-rank timed milliseconds (the job ends with its
@@ -147,432 +171,607 @@ def job_rate(units_per_rank_step, world, steps, max_ms):
     return units_per_rank_step * world * steps / (max_ms * 1e-3)
 
 
-# DRAM bytes (read + write) of one 4-bit launch of each headline kernel, measured with
-# ncu (--set full) on the 8192 x 8192 weight; scaled to a workload by element count.
-# Writes still dirty in L2 when a kernel ends are not in the DRAM count.
-NCU_DRAM_BYTES_8192SQ = {"qjl_v6": 134.53e6 + 25.83e6, "dequantize_v5": 34.65e6 + 74.65e6}
+def free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
 
 
-def alg_bytes_quant(n, bits):
-    return n * 2 + n * bits / 8 + 2 * n / D
+def relaunch_under_torchrun(args, argv):
+    """`--gpus N` started as a plain process: run N replicas, one per GPU, by
+    re-executing this script under torch.distributed.run (rank 0 prints)."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
-def alg_bytes_quant_qjl(n, bits):
-    return n * 2 + n * bits / 8 + 2 * n / D + n * M / (8 * D) + 2 * n / D
+# ---------------------------------------------------------------------------- workloads
+
+def make_llama(dev):
+    """The 32-layer input as one contiguous bf16 buffer (layer-major), matrix
+    i of the 224 drawn with seed 1000 + i."""
+    import torch
+    from kv_quantization_b200 import synth
+    x = torch.empty(LAYERS * LAYER_N, dtype=torch.bfloat16, device=dev)
+    off = 0
+    for i in range(LAYERS * len(LLAMA7B)):
+        r, c = LLAMA7B[i % len(LLAMA7B)]
+        x[off:off + r * c] = synth.llama_linear(r, c, seed=1000 + i, device=dev).reshape(-1)
+        off += r * c
+    return x
 
 
-def alg_bytes_dequant(n, bits):
-    return n * bits / 8 + 2 * n / D + n * 2
+def alg_quant(n, d=D, bits=BITS, m=0):
+    b = n * 2 + n * bits / 8 + 2 * n / d
+    if m:
+        b += n * m / (8 * d) + 2 * n / d
+    return b
 
 
-def run_device(args, rank, world):
+def alg_dequant(n, d=D, bits=BITS):
+    return n * bits / 8 + 2 * n / d + n * 2
+
+
+def ev():
+    import torch
+    return torch.cuda.Event(enable_timing=True)
+
+
+def l2_flusher(dev):
+    import torch
+    buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    return lambda: buf.view(torch.int32).sum()   # a 256 MB read evicts earlier data from the 126 MB L2
+
+
+# DRAM bytes (read + write) per launch from one-kernel ncu captures (profiles/):
+# the quantize and dequantize of one Llama-7B-shaped layer (202,375,168 values).
+NCU_DRAM_LAYER = {"quantize": None, "dequantize": None}
+
+
+def run_headline(args, dev, world, rank):
     import torch
     import kv_quantization_b200 as rq
-    from kv_quantization_b200 import synth
-
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    rq.lib()
-    x = make_inputs(dev)
+    cent = rq.rq_lloyd_max(BITS)
+    x = make_llama(dev)
     n = x.numel()
-    S = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
-    rq.qjl_make_projection(PROJ_SEED, M, D, S)
-    tabs = {b: rq.rq_lloyd_max(b) for b in BITS}
-    bufs = {}
-    for b in BITS:
-        bufs[b] = dict(
-            codes=torch.empty(rq.rq_code_bytes(n, D, b, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev),
-            norms=torch.empty(n // D, dtype=torch.int16, device=dev),
-            qs=torch.empty(n // D * M // 8, dtype=torch.uint8, device=dev),
-            qn=torch.empty(n // D, dtype=torch.int16, device=dev),
-            out=torch.empty_like(x))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    cb = LAYER_N * BITS // 8
+    codes = torch.empty(LAYERS * cb, dtype=torch.uint8, device=dev)
+    norms = torch.empty(n // D, dtype=torch.int16, device=dev)
+    out = torch.empty_like(x)
+    nb = LAYER_N // D
+    layer = [(x[l * LAYER_N:(l + 1) * LAYER_N], codes[l * cb:(l + 1) * cb], norms[l * nb:(l + 1) * nb],
+              out[l * LAYER_N:(l + 1) * LAYER_N]) for l in range(LAYERS)]
     stream = torch.cuda.current_stream()
-    n_ev = 2 * len(BITS)
-
-    def l2_flush():
-        flush.view(torch.int32).sum()   # read 256 MB: evicts earlier data from the 126 MB L2
 
     def step(evs=None):
-        # every kernel starts with a cold L2 (flush outside its event pair)
-        k = 0
-        for b in BITS:
-            B = bufs[b]
-            l2_flush()
-            if evs: evs[k][0].record(stream)
-            rq.rq_quantize_qjl(x, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], M, S, B["codes"], B["norms"],
-                               B["qs"], B["qn"])
-            if evs: evs[k][1].record(stream)
-            k += 1
-            l2_flush()
-            if evs: evs[k][0].record(stream)
-            rq.rq_dequantize(B["codes"], B["norms"], n, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], B["out"])
-            if evs: evs[k][1].record(stream)
-            k += 1
+        for l, (xl, cl, nl, ol) in enumerate(layer):
+            if evs: evs[2 * l][0].record(stream)
+            rq.rq_quantize(xl, D, BITS, rq.RQ_CODES_PACKED, 1, 1000 + l, cent, cl, nl)
+            if evs: evs[2 * l][1].record(stream)
+            if evs: evs[2 * l + 1][0].record(stream)
+            rq.rq_dequantize(cl, nl, LAYER_N, D, BITS, rq.RQ_CODES_PACKED, 1, 1000 + l, cent, ol)
+            if evs: evs[2 * l + 1][1].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-
-    kern_ms = [[0.0] * n_ev for _ in range(args.steps)]
-    step_ms = []
+    n_ev = 2 * LAYERS
+    evs_all = [[(ev(), ev()) for _ in range(n_ev)] for _ in range(args.steps)]
     clk = Clocks(dev.index)
     clk.start()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
     t0 = time.time()
-    evs_all = []
+    e0.record(stream)
     for s in range(args.steps):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
-        step(evs)
-        evs_all.append(evs)
+        step(evs_all[s])
+    e1.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
     if world > 1:
         dist.barrier()
     clk.window(t0, t1)
     clk.stop()
-    for s, evs in enumerate(evs_all):
-        for k in range(n_ev):
-            kern_ms[s][k] = evs[k][0].elapsed_time(evs[k][1])
-        step_ms.append(sum(kern_ms[s]))
-    total_ms = reduce_max_ms(sum(step_ms), world, dev)
-    in_bytes = n * 2 * len(BITS)
+    total_ms = reduce_max_ms(e0.elapsed_time(e1), world, dev)
+    q_ms = [evs_all[s][2 * l][0].elapsed_time(evs_all[s][2 * l][1]) for s in range(args.steps) for l in range(LAYERS)]
+    dq_ms = [evs_all[s][2 * l + 1][0].elapsed_time(evs_all[s][2 * l + 1][1])
+             for s in range(args.steps) for l in range(LAYERS)]
+    torch.cuda.synchronize()
+    assert rq.rq_device_error(True) == 0
+    in_bytes = n * 2
     value = job_rate(in_bytes, world, args.steps, total_ms) / 1e9
-    hbm, tf, src = peaks()
-    # dominant kernel: the larger of quantize_qjl / dequantize by total time
-    q_ms = [statistics.mean(kern_ms[s][2 * i] for s in range(args.steps)) for i in range(len(BITS))]
-    dq_ms = [statistics.mean(kern_ms[s][2 * i + 1] for s in range(args.steps)) for i in range(len(BITS))]
+    mq, mdq = statistics.mean(q_ms), statistics.mean(dq_ms)
     if sum(q_ms) >= sum(dq_ms):
-        dom, alg, ms = "qjl_v6_quant_kernel<b,bf16,signs> (d=128)", sum(alg_bytes_quant_qjl(n, b) for b in BITS), sum(q_ms)
-        traffic = NCU_DRAM_BYTES_8192SQ["qjl_v6"] * n / 8192 ** 2
+        dom = roofline_hbm(alg_quant(LAYER_N), mq, NCU_DRAM_LAYER["quantize"],
+                           kernel="quantize_v5_kernel<4,bf16,signs> (d=128)",
+                           alg_bytes_per_launch=alg_quant(LAYER_N), launches_timed=len(q_ms))
     else:
-        dom, alg, ms = "dequantize_v5_kernel<b,bf16,signs> (d=128)", sum(alg_bytes_dequant(n, b) for b in BITS), sum(dq_ms)
-        traffic = NCU_DRAM_BYTES_8192SQ["dequantize_v5"] * n / 8192 ** 2
-    achieved = alg / (ms * 1e-3) / 1e9
-    per_kernel = {f"quantize_qjl_b{b}_ms": round(q, 4) for b, q in zip(BITS, q_ms)}
-    per_kernel.update({f"dequantize_b{b}_ms": round(q, 4) for b, q in zip(BITS, dq_ms)})
-    per_kernel.update({f"quantize_qjl_b{b}_gbs": round(alg_bytes_quant_qjl(n, b) / (q * 1e-3) / 1e9, 1)
-                       for b, q in zip(BITS, q_ms)})
-    per_kernel.update({f"dequantize_b{b}_gbs": round(alg_bytes_dequant(n, b) / (q * 1e-3) / 1e9, 1)
-                       for b, q in zip(BITS, dq_ms)})
-
-    # quantize + dequantize alone (no QJL stage), same workload and cold L2
-    qd = {}
-    for b in BITS:
-        B = bufs[b]
-        tq, tdq = [], []
-        for _ in range(max(5, min(args.steps, 50))):
-            l2_flush()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            rq.rq_quantize(x, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], B["codes"], B["norms"])
-            e1.record(stream)
-            l2_flush()
-            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e2.record(stream)
-            rq.rq_dequantize(B["codes"], B["norms"], n, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], B["out"])
-            e3.record(stream)
-            torch.cuda.synchronize()
-            tq.append(e0.elapsed_time(e1))
-            tdq.append(e2.elapsed_time(e3))
-        mq, mdq = statistics.mean(tq), statistics.mean(tdq)
-        qd[f"b{b}"] = {"quantize_ms": round(mq, 4), "dequantize_ms": round(mdq, 4),
-                       "quantize_gbs": round(alg_bytes_quant(n, b) / (mq * 1e-3) / 1e9, 1),
-                       "dequantize_gbs": round(alg_bytes_dequant(n, b) / (mdq * 1e-3) / 1e9, 1),
-                       "input_gbs": round(n * 2 / ((mq + mdq) * 1e-3) / 1e9, 1),
-                       "pct_hbm": round(100 * (alg_bytes_quant(n, b) + alg_bytes_dequant(n, b)) /
-                                        ((mq + mdq) * 1e-3) / 1e9 / peaks()[0], 1)}
-
-    # end to end through the public API with host buffers
-    e2e = e2e_measure(args, x, S, tabs, bufs, dev)
-    secondary = [] if args.no_secondary else secondary_scores(dev)
-    result = {
+        dom = roofline_hbm(alg_dequant(LAYER_N), mdq, NCU_DRAM_LAYER["dequantize"],
+                           kernel="dequantize_v5_kernel<4,bf16,signs> (d=128)",
+                           alg_bytes_per_launch=alg_dequant(LAYER_N), launches_timed=len(dq_ms))
+    dom["traffic_note"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch on one layer "
+                           "(profiles/); null when not captured for this build")
+    pair = roofline_hbm(alg_quant(LAYER_N) + alg_dequant(LAYER_N), mq + mdq)
+    res = {
         "metric": "quantize+dequantize input GB/s", "value": round(value, 2), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 in, fp32 arithmetic", "data": "synthetic (seeded)",
-        "config": {"workload": WORKLOAD, "elements": n, "d": D, "bits": list(BITS), "qjl_m": M,
-                   "l2": "flushed (256 MB read) before every kernel; step time = sum of kernel times", "parallelism": f"replicas x{world}"},
-        "pct_hbm_peak": round(100 * achieved / hbm, 1),
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "peak_source": src, "traffic": round(traffic),
-                     "traffic_note": "ncu dram read+write of the 4-bit launch on the 8192^2 weight, scaled by "
-                                     "elements; per launch (achieved covers the 3-bit, 4-bit and 5-bit launches)",
-                     "alg_bytes_per_launch_4bit": round(alg_bytes_quant_qjl(n, 4) if dom.startswith("qjl")
-                                                        else alg_bytes_dequant(n, 4)),
-                     "alg_bytes_per_step": alg},
-        "kernels": per_kernel,
-        "quantize_dequantize_only": qd,
-        "e2e": e2e,
+        "vs_baseline": None, "dtype": "bf16 in/out, fp32 arithmetic, 4-bit codes", "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "elements": n, "d": D, "bits": BITS, "layers": LAYERS,
+                   "l2": "inputs (13 GB) far larger than L2; no flush needed",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "pct_hbm_peak": round(100 * pair["frac"], 1),
+        "roofline": dom,
+        "kernels": {"quantize_ms_per_layer": round(mq, 4), "dequantize_ms_per_layer": round(mdq, 4),
+                    "quantize": roofline_hbm(alg_quant(LAYER_N), mq),
+                    "dequantize": roofline_hbm(alg_dequant(LAYER_N), mdq),
+                    "pair": pair},
         "gpu_launches": n_ev * args.steps,
         "clocks": clk.summary(),
-        "secondary": secondary,
     }
-    return result
+    bufs = dict(x=x, codes=codes, norms=norms, out=out, cent=cent)
+    return res, bufs
 
 
-def e2e_measure(args, x, S, tabs, bufs, dev):
+def run_e2e(args, dev, bufs):
+    """The headline through the public API from pinned host buffers: per layer
+    the input goes host -> device, quantize + dequantize run, and the codes,
+    norms and reconstruction come back device -> host, pipelined over three
+    streams (copy in / compute / copy out) with two device buffers per role."""
     import torch
     import kv_quantization_b200 as rq
-    n = x.numel()
-    hx = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
-    hx.copy_(x.cpu())
-    hout = {b: {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in bufs[b].items()} for b in BITS}
-    dx = torch.empty_like(x)
-    stream = torch.cuda.current_stream()
-    bo = sum(v.numel() * v.element_size() for b in BITS for v in bufs[b].values())
+    x, cent = bufs["x"], bufs["cent"]
+    cb, nb = LAYER_N * BITS // 8, LAYER_N // D
+    try:
+        hx = torch.empty(x.numel(), dtype=torch.bfloat16, pin_memory=True)
+    except RuntimeError as e:
+        return {"unavailable": f"pinned host input buffer: {e}"}
+    hx.copy_(x)
+    x = None
+    bufs.clear()                      # the device copies of the headline are not needed any more
+    torch.cuda.empty_cache()
+    dxin = [torch.empty(LAYER_N, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dcodes = [torch.empty(cb, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dnorms = [torch.empty(nb, dtype=torch.int16, device=dev) for _ in range(2)]
+    dout = [torch.empty(LAYER_N, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    hout = [torch.empty(LAYER_N, dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    hcodes = [torch.empty(cb, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+    hnorms = [torch.empty(nb, dtype=torch.int16, pin_memory=True) for _ in range(2)]
+    s_in, s_c, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    main = torch.cuda.current_stream()
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    c_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        dx.copy_(hx, non_blocking=True)
-        for b in BITS:
-            B = bufs[b]
-            rq.rq_quantize_qjl(dx, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], M, S, B["codes"], B["norms"],
-                               B["qs"], B["qn"])
-            rq.rq_dequantize(B["codes"], B["norms"], n, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, tabs[b], B["out"])
-            for k, v in B.items():
-                hout[b][k].copy_(v, non_blocking=True)
+    def one_step():
+        s_in.wait_stream(main)
+        s_c.wait_stream(main)
+        s_out.wait_stream(main)
+        for l in range(LAYERS):
+            b = l & 1
+            with torch.cuda.stream(s_in):
+                if l >= 2:
+                    s_in.wait_event(c_done[b])               # compute of layer l-2 has read dxin[b]
+                dxin[b].copy_(hx[l * LAYER_N:(l + 1) * LAYER_N], non_blocking=True)
+                in_done[b].record(s_in)
+            with torch.cuda.stream(s_c):
+                s_c.wait_event(in_done[b])
+                if l >= 2:
+                    s_c.wait_event(out_done[b])              # layer l-2's results have left the device
+                rq.rq_quantize(dxin[b], D, BITS, rq.RQ_CODES_PACKED, 1, 1000 + l, cent, dcodes[b], dnorms[b],
+                               stream=s_c)
+                rq.rq_dequantize(dcodes[b], dnorms[b], LAYER_N, D, BITS, rq.RQ_CODES_PACKED, 1, 1000 + l, cent,
+                                 dout[b], stream=s_c)
+                c_done[b].record(s_c)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(c_done[b])
+                hout[b].copy_(dout[b], non_blocking=True)
+                hcodes[b].copy_(dcodes[b], non_blocking=True)
+                hnorms[b].copy_(dnorms[b], non_blocking=True)
+                out_done[b].record(s_out)
+        main.wait_stream(s_in)
+        main.wait_stream(s_c)
+        main.wait_stream(s_out)
 
-    for _ in range(2):
-        one()
+    one_step()
     torch.cuda.synchronize()
-    steps = max(3, min(args.steps, 10))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    steps = max(2, min(args.steps, 3))
+    e0, e1 = ev(), ev()
+    e0.record(main)
     for _ in range(steps):
-        one()
-    e1.record(stream)
+        one_step()
+    e1.record(main)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    return {"value": round(n * 2 * len(BITS) / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": n * 2, "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 4)}
+    h2d = LAYERS * LAYER_N * 2
+    d2h = LAYERS * (LAYER_N * 2 + cb + nb * 2)
+    return {"value": round(LAYERS * LAYER_N * 2 / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "path": "rq_quantize + rq_dequantize per layer, pinned host in/out, copies overlapped with compute"}
 
 
-def secondary_scores(dev, reps=5):
-    """QJL score tokens/s (key token-heads scored against all 32 queries per s)."""
+def median_ms(fn, reps, flush=None):
+    import torch
+    ts = []
+    for _ in range(reps):
+        if flush:
+            flush()
+        a, b = ev(), ev()
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def secondary_lines(dev, reps=10, only=None):
+    """Each secondary workload's kernels timed with CUDA events (median of
+    reps; L2 flushed before each rep where the input would fit in L2)."""
     import torch
     import kv_quantization_b200 as rq
     from kv_quantization_b200 import synth
+    flush = l2_flusher(dev)
     out = []
-    # KV cache 4 x 8 x 32768 x 128, K via QJL m = 256, pure QJL score
-    G, T, d, m, nq = 32, 32768, 128, 256, 32
-    k = synth.kv_with_channels(4, 8, T, d, seed=3, device=dev).reshape(-1)
-    S = torch.empty(m, d, dtype=torch.bfloat16, device=dev)
-    rq.qjl_make_projection(3, m, d, S)
-    signs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=dev)
-    kn = torch.empty(G * T, dtype=torch.int16, device=dev)
-    q = synth.normal((G, nq, d), seed=5, device=dev)
-    scores = torch.empty(G, nq, T, dtype=torch.float32, device=dev)
-    ws = torch.empty(rq.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=dev)
-    out.append(_time_pair("kv 4x8x32768x128 QJL m=256",
-                          lambda: rq.qjl_sketch(k, d, m, S, signs, kn),
-                          lambda: rq.qjl_score(q, G, nq, d, m, S, signs, kn, T, scores, ws), G * T,
-                          2 * m * d * G * T, k.numel() * 2 + signs.numel() + kn.numel() * 2, reps,
-                          score_bytes=signs.numel() + kn.numel() * 2 + 4 * G * nq * T))
-    del k, signs, kn, scores, ws
-    # TurboQuant-style 3-bit keys, head_dim 256: 2-bit + QJL m = d
-    G, T, d, bits = 8, 131072, 256, 2
-    m = d
-    k = synth.normal((G, T, d), seed=6, device=dev).reshape(-1)
-    cent = rq.rq_lloyd_max(bits)
-    S = torch.empty(m, d, dtype=torch.bfloat16, device=dev)
-    rq.qjl_make_projection(5, m, d, S)
-    codes = torch.empty(rq.rq_code_bytes(k.numel(), d, bits, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev)
-    norms = torch.empty(G * T, dtype=torch.int16, device=dev)
-    qs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=dev)
-    qn = torch.empty(G * T, dtype=torch.int16, device=dev)
-    q = synth.normal((G, nq, d), seed=7, device=dev)
-    scores = torch.empty(G, nq, T, dtype=torch.float32, device=dev)
-    ws = torch.empty(rq.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=dev)
-    out.append(_time_pair("keys 131072x8 d=256 2-bit+QJL m=d",
-                          lambda: rq.rq_quantize_qjl(k, d, bits, rq.RQ_CODES_PACKED, 1, 4, cent, m, S, codes, norms,
-                                                     qs, qn),
-                          lambda: rq.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms,
-                                               bits=bits, layout=rq.RQ_CODES_PACKED, use_signs=1, sign_seed=4,
-                                               centroids=cent),
-                          G * T, 2 * m * d * G * T, k.numel() * 2 + codes.numel() + qs.numel() + 4 * G * T, reps,
-                          score_bytes=codes.numel() + qs.numel() + 4 * G * T + 4 * G * nq * T))
-    del k, codes, norms, qs, qn, scores, ws
-    # the same at head_dim 512 (m = d = 512)
-    G, T, d, bits = 8, 131072, 512, 2
-    m = d
-    k = synth.normal((G, T, d), seed=8, device=dev).reshape(-1)
-    S = torch.empty(m, d, dtype=torch.bfloat16, device=dev)
-    rq.qjl_make_projection(9, m, d, S)
-    codes = torch.empty(rq.rq_code_bytes(k.numel(), d, bits, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev)
-    norms = torch.empty(G * T, dtype=torch.int16, device=dev)
-    qs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=dev)
-    qn = torch.empty(G * T, dtype=torch.int16, device=dev)
-    q = synth.normal((G, nq, d), seed=10, device=dev)
-    scores = torch.empty(G, nq, T, dtype=torch.float32, device=dev)
-    ws = torch.empty(rq.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=dev)
-    out.append(_time_pair("keys 131072x8 d=512 2-bit+QJL m=d",
-                          lambda: rq.rq_quantize_qjl(k, d, bits, rq.RQ_CODES_PACKED, 1, 4, cent, m, S, codes, norms,
-                                                     qs, qn),
-                          lambda: rq.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms,
-                                               bits=bits, layout=rq.RQ_CODES_PACKED, use_signs=1, sign_seed=4,
-                                               centroids=cent),
-                          G * T, 2 * m * d * G * T, k.numel() * 2 + codes.numel() + qs.numel() + 4 * G * T, reps,
-                          score_bytes=codes.numel() + qs.numel() + 4 * G * T + 4 * G * nq * T))
-    return out
+    want = (lambda k: True) if only is None else (lambda k: k == only)
 
+    if want("c1"):
+        # 256 x 512 fp16, d = 128, 4-bit int8 codes, no signs: L2-resident latency
+        x = synth.gaussian_matrix(256, 512, 0.02, seed=0, dtype=torch.float16, device=dev).reshape(-1)
+        cent = rq.rq_lloyd_max(4)
+        codes = torch.empty(x.numel(), dtype=torch.uint8, device=dev)
+        norms = torch.empty(x.numel() // 128, dtype=torch.int16, device=dev)
+        o = torch.empty_like(x)
+        q = lambda: rq.rq_quantize(x, 128, 4, rq.RQ_CODES_INT8, 0, 0, cent, codes, norms)
+        dq = lambda: rq.rq_dequantize(codes, norms, x.numel(), 128, 4, rq.RQ_CODES_INT8, 0, 0, cent, o)
+        q(); dq()
+        tq, tdq = median_ms(q, reps * 5), median_ms(dq, reps * 5)
+        out.append({"workload": "weight 256x512 fp16 N(0,0.02^2), d=128, 4-bit int8 codes, no signs",
+                    "quantize_us": round(tq * 1e3, 2), "dequantize_us": round(tdq * 1e3, 2),
+                    "round_trip_us": round((tq + tdq) * 1e3, 2), "note": "L2-resident; latency-bound (launch + one wave)"})
 
-def _time_pair(name, prep, score, tokens, prep_flops, prep_bytes, reps=5, score_bytes=None):
-    import torch
-    prep()
-    score()
+    if want("weight4096"):
+        x = synth.student_t_outliers(4096, 4096, seed=1, device=dev).reshape(-1)
+        n = x.numel()
+        m = 128
+        S = torch.empty(m, D, dtype=torch.bfloat16, device=dev)
+        rq.qjl_make_projection(2, m, D, S)
+        res = {"workload": "weight 4096x4096 bf16 student-t(4) std 0.02 + 0.1% outliers x20; d=128, signs seed 1; "
+                           "fused QJL residual sketch m=128 (S seed 2); bits 3/4/5", "l2": "flushed before each kernel"}
+        for b in (3, 4, 5):
+            cent = rq.rq_lloyd_max(b)
+            codes = torch.empty(rq.rq_code_bytes(n, D, b, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev)
+            norms = torch.empty(n // D, dtype=torch.int16, device=dev)
+            qs = torch.empty(n // D * m // 8, dtype=torch.uint8, device=dev)
+            qn = torch.empty(n // D, dtype=torch.int16, device=dev)
+            o = torch.empty_like(x)
+            fq = lambda: rq.rq_quantize_qjl(x, D, b, rq.RQ_CODES_PACKED, 1, 1, cent, m, S, codes, norms, qs, qn)
+            pq = lambda: rq.rq_quantize(x, D, b, rq.RQ_CODES_PACKED, 1, 1, cent, codes, norms)
+            dq = lambda: rq.rq_dequantize(codes, norms, n, D, b, rq.RQ_CODES_PACKED, 1, 1, cent, o)
+            fq(); dq()
+            tf_, tq, tdq = median_ms(fq, reps, flush), median_ms(pq, reps, flush), median_ms(dq, reps, flush)
+            res[f"b{b}"] = {"quantize_qjl_ms": round(tf_, 4), "quantize_ms": round(tq, 4), "dequantize_ms": round(tdq, 4),
+                            "input_gbs_fused_pair": round(n * 2 / ((tf_ + tdq) * 1e-3) / 1e9, 1),
+                            "input_gbs_pair": round(n * 2 / ((tq + tdq) * 1e-3) / 1e9, 1),
+                            "quantize_qjl_roofline": roofline_hbm(alg_quant(n, bits=b, m=m), tf_),
+                            "pair_roofline": roofline_hbm(alg_quant(n, bits=b) + alg_dequant(n, bits=b), tq + tdq)}
+        out.append(res)
+        del x, S
+
+    if want("kv_v"):
+        # V of the KV cache: RHT + 4-bit Lloyd-Max round trip
+        v = synth.kv_with_channels(4, 8, 32768, 128, seed=13, device=dev).reshape(-1)
+        n = v.numel()
+        cent = rq.rq_lloyd_max(4)
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        norms = torch.empty(n // 128, dtype=torch.int16, device=dev)
+        o = torch.empty_like(v)
+        q = lambda: rq.rq_quantize(v, 128, 4, rq.RQ_CODES_PACKED, 1, 14, cent, codes, norms)
+        dq = lambda: rq.rq_dequantize(codes, norms, n, 128, 4, rq.RQ_CODES_PACKED, 1, 14, cent, o)
+        q(); dq()
+        tq, tdq = median_ms(q, reps), median_ms(dq, reps)
+        out.append({"workload": "KV cache V 4x8x32768x128 bf16 N(0,1) (4 channels/head x10): RHT (signs seed 14) "
+                                "+ 4-bit Lloyd-Max quantize then dequantize",
+                    "quantize_ms": round(tq, 4), "dequantize_ms": round(tdq, 4),
+                    "input_gbs": round(n * 2 / ((tq + tdq) * 1e-3) / 1e9, 1),
+                    "roofline": roofline_hbm(alg_quant(n) + alg_dequant(n), tq + tdq)})
+        del v, codes, norms, o
+
+    if want("kv_k"):
+        G, T, d, m, nq = 32, 32768, 128, 256, 32
+        k = synth.kv_with_channels(4, 8, T, d, seed=3, device=dev).reshape(-1)
+        S = torch.empty(m, d, dtype=torch.bfloat16, device=dev)
+        rq.qjl_make_projection(3, m, d, S)
+        signs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=dev)
+        kn = torch.empty(G * T, dtype=torch.int16, device=dev)
+        q = synth.normal((G, nq, d), seed=5, device=dev)
+        scores = torch.empty(G, nq, T, dtype=torch.float32, device=dev)
+        ws = torch.empty(rq.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=dev)
+        sk = lambda: rq.qjl_sketch(k, d, m, S, signs, kn)
+        sc = lambda: rq.qjl_score(q, G, nq, d, m, S, signs, kn, T, scores, ws)
+        sk(); sc()
+        tk, ts = median_ms(sk, reps), median_ms(sc, reps, flush)
+        kbytes = k.numel() * 2 + signs.numel() + kn.numel() * 2
+        sbytes = signs.numel() + kn.numel() * 2 + 4 * G * nq * T
+        out.append({"workload": "KV cache K 4x8x32768x128 bf16 (4 channels/head x10): QJL sketch m=256 (S seed 3); "
+                                "pure-QJL score of 32 queries per (batch, head)",
+                    "sketch_ms": round(tk, 4), "score_ms": round(ts, 4),
+                    "score_tokens_per_s": round(G * T / (ts * 1e-3), 1),
+                    "sketch_roofline": roofline_hbm(kbytes, tk, flops=2 * m * d * G * T),
+                    "score_roofline": roofline_hbm(sbytes, ts, note="signs + norms read, fp32 scores written; "
+                                                                    "query prologue included")})
+        del k, signs, kn, scores, ws
+
+    for d, seed in ((256, 6), (512, 8)):
+        if not want(f"tq{d}"):
+            continue
+        G, T, bits, nq = 8, 131072, 2, 32
+        m = d
+        k = synth.normal((G, T, d), seed=seed, device=dev).reshape(-1)
+        cent = rq.rq_lloyd_max(bits)
+        S = torch.empty(m, d, dtype=torch.bfloat16, device=dev)
+        rq.qjl_make_projection(5, m, d, S)
+        codes = torch.empty(rq.rq_code_bytes(k.numel(), d, bits, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev)
+        norms = torch.empty(G * T, dtype=torch.int16, device=dev)
+        qs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=dev)
+        qn = torch.empty(G * T, dtype=torch.int16, device=dev)
+        q = synth.normal((G, nq, d), seed=7, device=dev)
+        scores = torch.empty(G, nq, T, dtype=torch.float32, device=dev)
+        ws = torch.empty(rq.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=dev)
+        cp = lambda: rq.rq_quantize_qjl(k, d, bits, rq.RQ_CODES_PACKED, 1, 4, cent, m, S, codes, norms, qs, qn)
+        sc = lambda: rq.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits,
+                                  layout=rq.RQ_CODES_PACKED, use_signs=1, sign_seed=4, centroids=cent)
+        cp(); sc()
+        tc, ts = median_ms(cp, reps), median_ms(sc, reps, flush)
+        n = k.numel()
+        cbytes = alg_quant(n, d=d, bits=bits, m=m)
+        flops = 2 * m * d * G * T
+        _, tf, _ = peaks()
+        hbm = peaks()[0]
+        tensor_bound = flops / cbytes > tf * 1e12 / (hbm * 1e9)
+        sbytes = codes.numel() + qs.numel() + 4 * G * T + 4 * G * nq * T
+        out.append({"workload": f"TurboQuant-style keys 131072 x 8 heads, d={d}, bf16 N(0,1): 2-bit (signs seed 4) + "
+                                f"QJL m={m} residual (S seed 5); score of 32 queries per head",
+                    "compress_ms": round(tc, 4), "score_ms": round(ts, 4),
+                    "score_tokens_per_s": round(G * T / (ts * 1e-3), 1),
+                    "compress_roofline": (roofline_tensor(flops, tc) if tensor_bound else
+                                          roofline_hbm(cbytes, tc, flops=flops)),
+                    "score_roofline": roofline_hbm(sbytes, ts, note="codes + signs + norms read, fp32 scores "
+                                                                    "written; query prologue included")})
+        del k, codes, norms, qs, qn, scores, ws
     torch.cuda.synchronize()
-    res = {"workload": name}
-    if reps <= 1:
-        return res
-    for label, fn in (("compress", prep), ("score", score)):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            fn()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / reps
-        res[f"{label}_ms"] = round(ms, 4)
-    res["score_tokens_per_s"] = round(tokens / (res["score_ms"] * 1e-3), 1)
-    res["compress_gbs"] = round(prep_bytes / (res["compress_ms"] * 1e-3) / 1e9, 1)
-    res["compress_tflops"] = round(prep_flops / (res["compress_ms"] * 1e-3) / 1e12, 2)
-    hbm, tf, src = peaks()
-    # compress: HBM-bound below the ridge (2 m d flops against 2 d + m/8 + ... bytes per vector)
-    ridge = tf * 1e12 / (hbm * 1e9)
-    if prep_flops / prep_bytes < ridge:
-        res["compress_roofline"] = {"bound": "hbm", "achieved": res["compress_gbs"], "peak": hbm, "unit": "GB/s",
-                                    "frac": round(res["compress_gbs"] / hbm, 4)}
-    else:
-        res["compress_roofline"] = {"bound": "tensor", "achieved": res["compress_tflops"], "peak": tf,
-                                    "unit": "TFLOP/s", "frac": round(res["compress_tflops"] / tf, 4)}
-    if score_bytes:
-        gbs = score_bytes / (res["score_ms"] * 1e-3) / 1e9
-        res["score_roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                                 "frac": round(gbs / hbm, 4),
-                                 "note": "packed keys + norms read, fp32 scores written; prologue included"}
-    return res
+    assert rq.rq_device_error(True) == 0
+    return out
 
 
 # ---------------------------------------------------------------------------- oracle arm
 
-def oracle_sample(n_blocks, seed=1):
-    """A bounded sample of the same workload for the CPU oracle: the first
-    n_blocks blocks of the seeded matrix (generated on the CPU)."""
-    import torch
+def cpu_info():
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count()
+
+
+def oracle_llama_sample(frac=8):
+    """The first 1/frac of each of layer 0's seven matrices (the same seeded
+    values the device arm quantizes), as bf16 bit patterns."""
     from kv_quantization_b200 import synth
-    x = synth.student_t_outliers(ROWS, COLS, seed=seed, device="cpu").reshape(-1)[: n_blocks * D]
-    return synth.as_u16(x).reshape(-1)
+    parts = []
+    for i, (r, c) in enumerate(LLAMA7B):
+        w = synth.llama_linear(r, c, seed=1000 + i, device="cpu").reshape(-1)
+        parts.append(synth.as_u16(w[: (r * c // frac) // D * D]).reshape(-1))
+    return np.concatenate(parts)
 
 
-def oracle_step(x16):
+def oracle_pair(x16, seed=1000):
     import oracle as O
-    s = O.sign_diagonal(SIGN_SEED, D)
-    S = O.projection(PROJ_SEED, M, D, O.BF16)
-    for b in BITS:
-        c = O.f32_table(b)
-        codes, norms, _, _ = O.quantize(x16, O.BF16, D, b, O.PACKED, s, c)
-        r, rn = O.residual(x16, O.BF16, codes, norms, D, b, O.PACKED, s, c)
-        O.sketch(r, O.BF16, D, M, S)
-        O.dequantize(codes, norms, D, b, O.PACKED, s, c, O.BF16)
+    s = O.sign_diagonal(seed, D)
+    c = O.f32_table(BITS)
+    codes, norms, _, _ = O.quantize(x16, O.BF16, D, BITS, O.PACKED, s, c)
+    O.dequantize(codes, norms, D, BITS, O.PACKED, s, c, O.BF16)
 
 
-def cpu_baseline(target_s=12.0):
+def cpu_baseline():
+    """The oracle (single-threaded C), as it stands, on bounded samples: the
+    headline's metric on a sample of the headline workload, plus one timing
+    per secondary workload."""
+    import torch
     import oracle as O
+    from kv_quantization_b200 import synth
     O.lib()
-    x16 = oracle_sample(64)
+    model, ncpu = cpu_info()
+    x16 = oracle_llama_sample()
     t0 = time.perf_counter()
-    oracle_step(x16)
-    per_block = (time.perf_counter() - t0) / 64
-    nb = int(max(64, min(ROWS * COLS // D, target_s / max(per_block, 1e-9))))
-    x16 = oracle_sample(nb)
-    t0 = time.perf_counter()
-    oracle_step(x16)
+    oracle_pair(x16)
     dt = time.perf_counter() - t0
-    return {"value": round(nb * D * 2 * len(BITS) / dt / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {nb} of {ROWS * COLS // D} blocks of the same matrix, bits 3/4/5, "
-                      f"quantize+residual+sketch+dequantize, {dt:.1f} s single-threaded C"}
+    res = {"value": round(x16.size * 2 / dt / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"first 1/8 of each of layer 0's seven matrices ({x16.size} values), 4-bit quantize + "
+                     f"dequantize, {dt:.1f} s on one thread",
+           "cpu_model": model, "nproc": ncpu, "per_workload": {}}
+    pw = res["per_workload"]
+    # weight 256x512 fp16 (whole)
+    w = synth.gaussian_matrix(256, 512, 0.02, seed=0, dtype=torch.float16, device="cpu").reshape(-1)
+    w16 = synth.as_u16(w).reshape(-1)
+    c4 = O.f32_table(4)
+    t0 = time.perf_counter()
+    cds, nrm, _, _ = O.quantize(w16, O.F16, 128, 4, O.INT8, None, c4)
+    O.dequantize(cds, nrm, 128, 4, O.INT8, None, c4, O.F16)
+    pw["weight256x512_round_trip_us"] = round((time.perf_counter() - t0) * 1e6, 1)
+    # weight 4096^2 fused 4-bit, first 4096 blocks
+    x = synth.student_t_outliers(4096, 4096, seed=1, device="cpu").reshape(-1)[: 4096 * 128]
+    x16 = synth.as_u16(x).reshape(-1)
+    S = O.projection(2, 128, 128, O.BF16)
+    s = O.sign_diagonal(1, 128)
+    t0 = time.perf_counter()
+    cds, nrm, _, _ = O.quantize(x16, O.BF16, 128, 4, O.PACKED, s, c4)
+    r, rn = O.residual(x16, O.BF16, cds, nrm, 128, 4, O.PACKED, s, c4)
+    O.sketch(r, O.BF16, 128, 128, S)
+    dt = time.perf_counter() - t0
+    pw["weight4096_fused_b4_gbs"] = round(x16.size * 2 / dt / 1e9, 6)
+    # KV keys: sketch of 16384 keys, score of 32 queries over 4096 keys
+    k = synth.kv_with_channels(1, 1, 16384, 128, seed=3, device="cpu").reshape(-1)
+    k16 = synth.as_u16(k).reshape(-1)
+    S = O.projection(3, 256, 128, O.BF16)
+    t0 = time.perf_counter()
+    sg, _ = O.sketch(k16, O.BF16, 128, 256, S)
+    dt = time.perf_counter() - t0
+    pw["kv_sketch_keys_per_s"] = round(16384 / dt, 1)
+    kn = O.vec_norms(k16, O.BF16, 128)
+    q16 = synth.as_u16(synth.normal((1, 32, 128), seed=5, device="cpu")).reshape(-1)
+    t0 = time.perf_counter()
+    O.score(q16, 1, 32, 128, 256, S, O.BF16, sg[: 4096 * 32], kn[:4096], 4096)
+    pw["kv_score_token_heads_per_s"] = round(4096 / (time.perf_counter() - t0), 1)
+    # TurboQuant-style keys at d = 256 / 512: compress 2048 keys, score 32 queries over 2048 keys
+    for d in (256, 512):
+        kk = synth.normal((1, 2048, d), seed=6, device="cpu").reshape(-1)
+        kk16 = synth.as_u16(kk).reshape(-1)
+        c2 = O.f32_table(2)
+        sd = O.sign_diagonal(4, d)
+        S = O.projection(5, d, d, O.BF16)
+        t0 = time.perf_counter()
+        cds, nrm, _, _ = O.quantize(kk16, O.BF16, d, 2, O.PACKED, sd, c2)
+        r, rn = O.residual(kk16, O.BF16, cds, nrm, d, 2, O.PACKED, sd, c2)
+        sg, _ = O.sketch(r, O.BF16, d, d, S)
+        pw[f"tq{d}_compress_keys_per_s"] = round(2048 / (time.perf_counter() - t0), 1)
+        q16 = synth.as_u16(synth.normal((1, 32, d), seed=7, device="cpu")).reshape(-1)
+        t0 = time.perf_counter()
+        O.score(q16, 1, 32, d, d, S, O.BF16, sg, rn, 2048, codes=cds, norms=nrm, bits=2, layout=O.PACKED,
+                signs_diag=sd, c32=c2)
+        pw[f"tq{d}_score_token_heads_per_s"] = round(2048 / (time.perf_counter() - t0), 1)
+    return res
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step a bounded sample of the workload."""
+    """The oracle as the reference arm, on the headline's metric and workload:
+    each step a bounded sample (the first 1/64 of each of layer 0's matrices)."""
     import oracle as O
     O.lib()
-    nb = 256
-    x16 = oracle_sample(nb)
+    x16 = oracle_llama_sample(frac=64)
     for _ in range(args.warmup):
-        oracle_step(x16)
+        oracle_pair(x16)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(x16)
+        oracle_pair(x16)
     dt = time.perf_counter() - t0
-    v = nb * D * 2 * len(BITS) * args.steps / dt / 1e9
+    v = x16.size * 2 * args.steps / dt / 1e9
+    model, ncpu = cpu_info()
+    sample = f"first 1/64 of each of layer 0's seven matrices ({x16.size} values) per step"
     return {"impl": "reference", "metric": "quantize+dequantize input GB/s", "value": round(v, 6), "unit": "GB/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32/fp64 arithmetic",
-            "data": "synthetic (seeded)",
-            "config": {"workload": WORKLOAD, "sample_blocks_per_step": nb},
-            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{nb} blocks of the workload per step"},
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in/out, fp32 arithmetic (fp64 where the oracle fixes it), 4-bit codes",
+            "data": "synthetic (seeded)", "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                             "cpu_model": model, "nproc": ncpu},
             "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def kernels_once():
-    """Each hot kernel once, inputs larger than L2: 8192 x 8192 bf16 weight
-    (quantize, quantize+QJL, dequantize at 4 bits), the 4 x 8 x 32768 x 128 KV
-    cache (QJL sketch m=256 and its score), 131072 x 8 keys at head_dim 256
-    (2-bit + QJL m=d and its score)."""
+# ---------------------------------------------------------------------------- profiling driver
+
+def profile_case(case):
+    """Run one case's kernels once on inputs larger than L2 (for one-kernel ncu
+    captures); prints nothing."""
     import torch
     import kv_quantization_b200 as rq
     from kv_quantization_b200 import synth
     dev = torch.device("cuda:0")
-    x = synth.student_t_outliers(8192, 8192, seed=1, device=dev).reshape(-1)
-    n, b = x.numel(), 4
-    cent = rq.rq_lloyd_max(b)
-    S = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
-    rq.qjl_make_projection(PROJ_SEED, M, D, S)
-    codes = torch.empty(rq.rq_code_bytes(n, D, b, rq.RQ_CODES_PACKED), dtype=torch.uint8, device=dev)
-    norms = torch.empty(n // D, dtype=torch.int16, device=dev)
-    qs = torch.empty(n // D * M // 8, dtype=torch.uint8, device=dev)
-    qn = torch.empty(n // D, dtype=torch.int16, device=dev)
-    out = torch.empty_like(x)
-    rq.rq_quantize(x, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, cent, codes, norms)
-    rq.rq_quantize_qjl(x, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, cent, M, S, codes, norms, qs, qn)
-    rq.rq_dequantize(codes, norms, n, D, b, rq.RQ_CODES_PACKED, 1, SIGN_SEED, cent, out)
-    del x, out
-    secondary_scores(dev, reps=1)
+    if case == "c3_layer":
+        x = torch.empty(LAYER_N, dtype=torch.bfloat16, device=dev)
+        off = 0
+        for i, (r, c) in enumerate(LLAMA7B):
+            x[off:off + r * c] = synth.llama_linear(r, c, seed=1000 + i, device=dev).reshape(-1)
+            off += r * c
+        cent = rq.rq_lloyd_max(BITS)
+        codes = torch.empty(LAYER_N * BITS // 8, dtype=torch.uint8, device=dev)
+        norms = torch.empty(LAYER_N // D, dtype=torch.int16, device=dev)
+        out = torch.empty_like(x)
+        rq.rq_quantize(x, D, BITS, rq.RQ_CODES_PACKED, 1, 1000, cent, codes, norms)
+        rq.rq_dequantize(codes, norms, LAYER_N, D, BITS, rq.RQ_CODES_PACKED, 1, 1000, cent, out)
+    else:
+        key = {"weight4096_fused": "weight4096", "kv_sketch": "kv_k", "kv_score": "kv_k", "kv_v": "kv_v",
+               "tq256": "tq256", "tq512": "tq512"}[case]
+        secondary_lines(dev, reps=1, only=key)
     torch.cuda.synchronize()
     assert rq.rq_device_error(True) == 0
 
 
-def main():
-    args = parse()
-    if args.kernels_once:
-        kernels_once()
-        return
+# ---------------------------------------------------------------------------- main
+
+def rank_selftest(args, rank, world):
+    """CPU stand-in for the device arm, used by the multi-rank tests: each
+    rank 'times' a fixed amount of work so that the launcher, the barrier and
+    the max-over-ranks aggregation can be checked without a GPU."""
+    local_ms = 10.0 * (rank + 1)
+    total_ms = reduce_max_ms(local_ms * args.steps, world)
+    return {"metric": "rank selftest units/s", "value": job_rate(100.0, world, args.steps, total_ms),
+            "unit": "units/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps}
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse(argv)
+    if args.profile:
+        profile_case(args.profile)
+        return 0
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_under_torchrun(args, argv)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
+    if world != args.gpus:
+        print(json.dumps({"error": f"WORLD_SIZE={world} but --gpus {args.gpus}"}), flush=True)
+        return 2
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
-        return
+        return 0
     if world > 1:
         import datetime
-        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    res = run_device(args, rank, world)
+        if args.rank_selftest:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        else:
+            import torch
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.rank_selftest:
+        res = rank_selftest(args, rank, world)
+    else:
+        import torch
+        import kv_quantization_b200 as rq
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(dev)
+        rq.lib()
+        res, bufs = run_headline(args, dev, world, rank)
+        # every rank takes the same remaining steps (no collectives in them)
+        res["e2e"] = {"skipped": "--no-e2e"} if args.no_e2e else run_e2e(args, dev, bufs)
+        del bufs
+        torch.cuda.empty_cache()
+        res["secondary"] = [] if args.no_secondary else secondary_lines(dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
     if rank == 0:
-        if not args.no_cpu:
+        if not args.no_cpu and not args.rank_selftest:
             res["cpu_baseline"] = cpu_baseline()
         print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -32,9 +32,10 @@
  *     returns.  Kernel faults surface at the caller's next synchronisation.
  *   - Return value: RQ_OK or a negative rq_status; on error nothing is enqueued.
  *   - Device pointers must be 16-byte aligned.
- *   - d (block size / head dim) is a power of two in {64, 128, 256, 512}
- *     ("--block-size N, must be a power of 2" and "head_dim must be a power of
- *     2" on the pages); n must be a multiple of d.
+ *   - d (block size / head dim) is a power of two in {64, 128, 256, 512}: the
+ *     PolarQuant section's knob list restricts its block size to powers of two,
+ *     and the Fused TurboQuant section's compatibility constraints restrict the
+ *     butterfly Hadamard to power-of-two head dims.  n must be a multiple of d.
  *   - Arithmetic is fp32 in one canonical order so results are reproducible
  *     bit for bit: the norm is the pairwise (recursive halving) fp32 sum of
  *     fp32 squares with a correctly rounded sqrt; the Hadamard transform runs
@@ -87,15 +88,35 @@ const char *rq_status_string(int status);
  * Returns RQ_ECUDA if the word cannot be read. */
 rq_status rq_device_error(int clear);
 
+/* Launch trace: the names of the kernels that the last librq call made on
+ * the calling host thread enqueued, comma-separated in launch order (e.g.
+ * "score_v2_prologue,score_v4_kernel"), or "" when that call returned an error
+ * before enqueuing anything.  Thread-local storage owned by the library, valid
+ * until the thread's next librq call.  Which kernel runs is chosen from the
+ * shape (d, bits, m, n_q, shared-memory fit); this lets a caller or a test see
+ * the choice. */
+const char *rq_last_launch(void);
+
+/* Self-test of the bounded-wait failure path (no counterpart on the pages; it
+ * exercises the loud-failure behaviour the entry points promise).  Enqueues
+ * one CTA that allocates tensor memory, waits at most `polls` times (1 ..
+ * 2^20) on an mbarrier that nothing ever arrives on, then unwinds exactly as
+ * the tensor-core kernels do after an expired wait: it records RQ_EDEVICE in
+ * the device error word, frees its tensor memory and returns.  No copy or MMA
+ * is in flight while it waits.  After it completes, rq_device_error() reports
+ * RQ_EDEVICE until cleared; the device stays usable.  RQ_EINVAL for polls out
+ * of range. */
+rq_status rq_probe_bounded_wait(uint32_t polls, rq_stream_t stream);
+
 /* Bytes of code storage for n values in blocks of d: (n/d) * (d*bits/8) packed,
  * n for int8.  Returns -1 on invalid arguments. */
 int64_t rq_code_bytes(int64_t n, int d, int bits, rq_layout layout);
 
 /* Lloyd-Max reconstruction levels for N(0,1) at `bits` (1..8), ascending,
  * written to the HOST array centroids_out[2^bits] as fp32.  Computed by the
- * conditional-expectation fixed point in fp64 (PolarQuant paragraph: "Lloyd-Max
- * optimal centroids for N(0,1) ... iterative conditional-expectation
- * algorithm"), made exactly odd-symmetric, then rounded to fp32. */
+ * conditional-expectation fixed point in fp64 (the PolarQuant paragraph's
+ * optimal N(0,1) levels found by iterating conditional means), made exactly
+ * odd-symmetric, then rounded to fp32. */
 rq_status rq_lloyd_max(int bits, float *centroids_out);
 
 /* Quantize n values of x (dtype fp16/bf16, n % d == 0, blocks contiguous).
@@ -116,8 +137,8 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
                         void *out, rq_dtype out_dtype, rq_stream_t stream);
 
 /* Quantize (as rq_quantize) and sketch the first-stage residual in the same
- * pass (PolarQuant paragraph: "optionally append a 1-bit QJL residual"; the
- * two-stage TurboQuant-style key code):
+ * pass (the optional 1-bit QJL residual correction of the PolarQuant
+ * paragraph; the two-stage TurboQuant-style key code):
  *   r = x - x^32 (fp32, x^32 the reconstruction before output rounding),
  *   qjl_norms[b] = fp16(||r||) (canonical fp32 norm),
  *   qjl_signs[b][m/8] = sign bits of S r_bf16, r_bf16 = bf16(r), S = proj.
@@ -135,9 +156,9 @@ rq_status rq_quantize_qjl(const void *x, rq_dtype dtype, int64_t n, int d, int b
 rq_status qjl_make_projection(uint64_t seed, int m, int d, rq_dtype dtype, void *proj, rq_stream_t stream);
 
 /* QJL sketch of n_vec vectors x[n_vec][d] (dtype = proj dtype):
- * signs[n_vec][m/8] of S x, norms[n_vec] = fp16(||x||) (QJL paragraph:
- * "extract ||k||", "take the sign of each sketch coordinate, packing 8 signs
- * into one uint8"). */
+ * signs[n_vec][m/8] of S x, norms[n_vec] = fp16(||x||) (the QJL paragraph:
+ * the key's norm is kept, and the sign of every sketch coordinate is stored
+ * as one bit, eight to a byte). */
 rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m, const void *proj,
                      uint8_t *signs, uint16_t *norms, rq_stream_t stream);
 
@@ -172,8 +193,11 @@ rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void 
  *   - Returns RQ_ESIZE when qjl_score_workspace_bytes(G, n_q, d, m) exceeds
  *     8 MiB (8388608 bytes), before touching the GPU.
  *   - The first call on a device looks up the array's device address (with
- *     that device current) and remembers it; make that first call before any
- *     stream capture.  RQ_ECUDA if the lookup fails.
+ *     that device current) and remembers it together with the device's
+ *     current context; make that first call before any stream capture.  After
+ *     a device reset the next call sees a new context and looks the address up
+ *     again (that call, too, belongs before any capture).  RQ_ECUDA if the
+ *     lookup fails.
  *   - Every call on a device shares the one array and it keeps the last
  *     call's contents (nothing in it needs to start at zero).  Calls whose
  *     work overlaps on the GPU -- e.g. on two streams without ordering between

@@ -43,6 +43,8 @@ def lib() -> C.CDLL:
                 "rq_status_string": (C.c_char_p, [i32]),
                 "rq_code_bytes": (i64, [i64, i32, i32, i32]),
                 "rq_device_error": (i32, [i32]),
+                "rq_last_launch": (C.c_char_p, []),
+                "rq_probe_bounded_wait": (i32, [C.c_uint32, vp]),
                 "rq_lloyd_max": (i32, [i32, fp]),
                 "rq_quantize": (i32, [vp, i32, i64, i32, i32, i32, i32, u64, fp, vp, vp, vp]),
                 "rq_dequantize": (i32, [vp, vp, i64, i32, i32, i32, i32, u64, fp, vp, i32, vp]),
@@ -65,7 +67,7 @@ def lib() -> C.CDLL:
 
 def exported_symbols():
     """Names this binding expects librq.so to export."""
-    return ["rq_status_string", "rq_device_error", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
+    return ["rq_status_string", "rq_device_error", "rq_last_launch", "rq_probe_bounded_wait", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
             "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score",
             "qjl_score_noalloc"]
 
@@ -113,6 +115,15 @@ def rq_code_bytes(n: int, d: int, bits: int, layout: int) -> int:
 def rq_device_error(clear: bool = True) -> int:
     """RQ_OK, or RQ_EDEVICE when a kernel gave up a bounded wait since the last clear."""
     return lib().rq_device_error(int(clear))
+
+
+def rq_last_launch() -> str:
+    """Kernels enqueued by this thread's last librq call, comma-separated."""
+    return lib().rq_last_launch().decode()
+
+
+def rq_probe_bounded_wait(polls: int, stream=None):
+    _check("rq_probe_bounded_wait", lib().rq_probe_bounded_wait(int(polls), _stream(stream)))
 
 
 def rq_lloyd_max(bits: int) -> np.ndarray:

@@ -45,6 +45,7 @@ cudaError_t launch_projection(uint64_t seed, int m, int d, bool bf16, void *proj
     const int threads = 256;
     projection_kernel<<<(unsigned)((count + threads - 1) / threads), threads, 0, st>>>(
         seed, count, bf16, static_cast<uint16_t *>(proj));
+    note_launch("projection_kernel");
     return cudaGetLastError();
 }
 
@@ -184,6 +185,7 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
     const unsigned zsl = (unsigned)((sc2_m64(a.m) + kSc2PrologueOut - 1) / kSc2PrologueOut);   // 16 S q outputs per CTA
     score_v2_prologue<<<dim3((unsigned)a.G, (unsigned)((a.nq + kSc2PrologueQ - 1) / kSc2PrologueQ), zsl), 256, psmem, st>>>(
         a.q, a.nq, a.d, a.m, static_cast<const uint16_t *>(a.proj), a.proj_bf16, *a.tables, TWO, wsB, wsN);
+    note_launch("score_v2_prologue");
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t items = a.G * ((a.T + 127) / 128);
@@ -201,6 +203,7 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
             kern4<<<(unsigned)(grid > 0 ? grid : 1), kSc4Threads, smem4, st>>>(
                 wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms, a.T, a.G, a.codes, a.norms, *a.tables, a.scores, c.ring,
                 c.slc);
+            note_launch("score_v4_kernel");
             return cudaGetLastError();
         }
     }
@@ -218,6 +221,7 @@ static cudaError_t launch_score_main(const ScoreArgs &a, cudaStream_t st)
               (unsigned)((a.nq + kScoreQ - 1) / kScoreQ));
     kern<<<grid, kScoreThreads, smem, st>>>(a.workspace, a.nq, a.d, a.m, a.signs, a.sk_norms, a.T, a.codes,
                                             a.norms, *a.tables, a.scores);
+    note_launch("score_kernel");
     return cudaGetLastError();
 }
 
@@ -246,6 +250,7 @@ cudaError_t launch_score(const ScoreArgs &a, cudaStream_t st)
     const size_t psmem = (size_t)2 * a.d * sizeof(float);
     score_prologue_kernel<<<(unsigned)(a.G * a.nq), 256, psmem, st>>>(a.q, a.d, a.m, a.proj, a.proj_bf16, *a.tables,
                                                                       two, a.workspace);
+    note_launch("score_prologue_kernel");
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (!two) return launch_score_main<1, false>(a, st);

@@ -22,6 +22,24 @@ using rq::QuantTables;
 namespace rq {
 // Set (bitwise OR) by a kernel whose bounded wait on the tensor core expired.
 __device__ unsigned int g_device_error = 0;
+
+// Names of the kernels the calling thread's last entry-point call enqueued,
+// comma-separated (rq_last_launch).
+namespace {
+constexpr size_t kTraceBytes = 256;
+thread_local char g_trace[kTraceBytes];
+}  // namespace
+
+void begin_call() { g_trace[0] = '\0'; }
+
+void note_launch(const char *kernel)
+{
+    size_t n = std::strlen(g_trace);
+    const size_t k = std::strlen(kernel);
+    if (n + k + 2 > kTraceBytes) return;
+    if (n) g_trace[n++] = ',';
+    std::memcpy(g_trace + n, kernel, k + 1);
+}
 }  // namespace rq
 
 namespace {
@@ -405,6 +423,7 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
                                const void *proj, void *codes, uint16_t *norms, uint8_t *qjl_signs,
                                uint16_t *qjl_norms, cudaStream_t stream)
 {
+    rq::begin_call();
     rq_status s = check_common(n, d, bits, layout);
     if (s) return s;
     if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
@@ -455,6 +474,7 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
                         rq_layout layout, int use_signs, uint64_t sign_seed, const float *centroids,
                         void *out, rq_dtype out_dtype, rq_stream_t stream)
 {
+    rq::begin_call();
     rq_status s = check_common(n, d, bits, layout);
     if (s) return s;
     if (out_dtype != RQ_F16 && out_dtype != RQ_BF16) return RQ_EINVAL;
@@ -476,6 +496,7 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
 
 rq_status qjl_make_projection(uint64_t seed, int m, int d, rq_dtype dtype, void *proj, rq_stream_t stream)
 {
+    rq::begin_call();
     if (m < 8 || m > 512 || m % 8 || !pow2_d(d)) return RQ_EINVAL;
     if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
     if (!proj) return RQ_EINVAL;
@@ -487,6 +508,7 @@ rq_status qjl_make_projection(uint64_t seed, int m, int d, rq_dtype dtype, void 
 rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m, const void *proj,
                      uint8_t *signs, uint16_t *norms, rq_stream_t stream)
 {
+    rq::begin_call();
     if (!pow2_d(d)) return RQ_EINVAL;
     if (m < 8 || m > 512 || m % 8) return RQ_EINVAL;
     if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
@@ -505,6 +527,15 @@ rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m,
         a.has_tmap_s = (m16 <= 256 || m16 % 256 == 0) && rq::make_proj_tmap(&a.tmap_s, proj, m, d, m16 < 256 ? m16 : 256);
     }
     return cuda_status(rq::launch_sketch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char *rq_last_launch(void) { return rq::g_trace; }
+
+rq_status rq_probe_bounded_wait(uint32_t polls, rq_stream_t stream)
+{
+    rq::begin_call();
+    if (polls < 1 || polls > rq::kProbeMaxPolls) return RQ_EINVAL;
+    return cuda_status(rq::launch_wait_probe(polls, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rq_status rq_device_error(int clear)
@@ -530,6 +561,7 @@ rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void 
                     int use_signs, uint64_t sign_seed, const float *centroids,
                     float *scores, void *workspace, size_t workspace_bytes, rq_stream_t stream)
 {
+    rq::begin_call();
     if (!pow2_d(d)) return RQ_EINVAL;
     if (m < 8 || m > 512 || m % 8) return RQ_EINVAL;
     if (proj_dtype != RQ_F16 && proj_dtype != RQ_BF16) return RQ_EINVAL;

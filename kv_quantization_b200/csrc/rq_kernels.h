@@ -78,6 +78,12 @@ struct ScoreArgs {
     int num_sms;
 };
 
+// Launch trace of the calling host thread (rq_last_launch): begin_call()
+// empties it at the start of every entry point, note_launch() appends the
+// name of a kernel just enqueued.
+void begin_call();
+void note_launch(const char *kernel);
+
 cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st);
 cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t st);
 cudaError_t launch_projection(uint64_t seed, int m, int d, bool bf16, void *proj, cudaStream_t st);
@@ -95,5 +101,9 @@ bool make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d, int 
 // Encode S[m][d] (16-bit) with {64 columns, box_rows rows} boxes (B operand layout).
 bool make_proj_tmap(CUtensorMap *map, const void *ptr, int m, int d, int box_rows);
 size_t dequantize_smem_bytes(int d);
+// One CTA that waits, at most `polls` times, on an mbarrier nothing arrives
+// on, then unwinds as the tensor-core kernels do (rq_probe_bounded_wait).
+constexpr uint32_t kProbeMaxPolls = 1u << 20;
+cudaError_t launch_wait_probe(uint32_t polls, cudaStream_t st);
 
 }  // namespace rq

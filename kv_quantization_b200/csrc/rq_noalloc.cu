@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "rq.h"
@@ -28,18 +29,47 @@ static __device__ __align__(256) unsigned char g_score_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void *g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and remembered; nullptr on failure.
+// The driver's cuCtxGetCurrent, looked up once through the runtime (the
+// library links only against cudart).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CtxGetCurrentFn ctx_get_current()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    }
+    return fn;
+}
+
+// Device address of the scratch array on the current device, looked up with
+// that device current and remembered together with the context it belongs
+// to; nullptr on failure.  A device reset (or any teardown and re-creation of
+// the primary context) reloads the library's module, possibly at another
+// address: the context check sees the new context and looks the address up
+// again instead of handing out a stale pointer.
 void *scratch_for_current_device()
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return nullptr;
+    // The context current on this thread; null when the runtime has not made
+    // the device's primary context current here yet (the lookup below does).
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return nullptr;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
+    if (!ctx || !g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_score_scratch) != cudaSuccess || !p) return nullptr;
+        if (get(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     return g_scratch_ptr[dev];
 }

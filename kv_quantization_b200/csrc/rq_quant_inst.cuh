@@ -32,6 +32,7 @@ static cudaError_t launch_q(const QuantArgs &a, cudaStream_t st)
     kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
         static_cast<const uint8_t *>(a.x), a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms,
         a.m, static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
+    note_launch("quantize_kernel");
     return cudaGetLastError();
 }
 
@@ -51,6 +52,7 @@ static cudaError_t launch_mma(const QuantTables &T, const void *x, int64_t nvec,
     kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
         static_cast<const uint8_t *>(x), nvec, T, static_cast<uint8_t *>(codes), norms, m,
         static_cast<const uint16_t *>(proj), signs, snorms);
+    note_launch(MODE == 0 ? "qjl_mma_kernel<fused>" : "qjl_mma_kernel<sketch>");
     return cudaGetLastError();
 }
 
@@ -67,6 +69,7 @@ static cudaError_t launch_qjl_v3_ns(const QuantArgs &a, size_t smem, cudaStream_
     kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_v, a.nblocks, *a.tables,
                                                             static_cast<uint8_t *>(a.codes), a.norms, a.m,
                                                             static_cast<const uint16_t *>(a.proj), a.qsigns, a.qnorms);
+    note_launch("qjl_v3_quant_kernel");
     return cudaGetLastError();
 }
 
@@ -104,27 +107,7 @@ static cudaError_t launch_sketch_v3(const SketchArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(grid > 0 ? grid : 1), kSk3Warps * 32, smem, st>>>(a.tmap_k, a.tmap_s, a.nvec, a.m, a.signs,
                                                                         a.norms);
-    return cudaGetLastError();
-}
-
-template <bool BF16>
-static cudaError_t launch_sketch_v2(const SketchArgs &a, cudaStream_t st)
-{
-    if (!a.has_tmap_k || 2 * qjl_mma_m16(a.m) > 512) return cudaErrorNotSupported;
-    QuantTables T{};
-    size_t smem = qjl_v2_smem(1, 1, a.m, T, 5);
-    auto kern = qjl_v2_sketch_kernel<BF16, 5>;
-    if (smem > kMaxSmemPerBlock) {
-        smem = qjl_v2_smem(1, 1, a.m, T, 3);
-        kern = qjl_v2_sketch_kernel<BF16, 3>;
-    }
-    if (smem > kMaxSmemPerBlock) return cudaErrorNotSupported;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int64_t tiles = (a.nvec + 127) / 128;
-    const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
-    kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_k, a.nvec, a.m,
-                                                            static_cast<const uint16_t *>(a.proj), a.signs, a.norms);
+    note_launch("sketch_v3_kernel");
     return cudaGetLastError();
 }
 
@@ -144,6 +127,7 @@ static cudaError_t launch_q2(const QuantArgs &a, cudaStream_t st)
     const int64_t grid = tiles < cap ? tiles : cap;
     kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(a.tmap_x, rows, *a.tables,
                                                             static_cast<uint8_t *>(a.codes), a.norms);
+    note_launch("quantize_v2_kernel");
     return cudaGetLastError();
 }
 
@@ -163,6 +147,7 @@ static cudaError_t launch_dq2(const DequantArgs &a, cudaStream_t st)
     const int64_t grid = tiles < cap ? tiles : cap;
     kern<<<(unsigned)(grid > 0 ? grid : 1), kT2, smem, st>>>(static_cast<const uint8_t *>(a.codes), a.norms, rows,
                                                             *a.tables, a.tmap_out);
+    note_launch("dequantize_v2_kernel");
     return cudaGetLastError();
 }
 
@@ -181,6 +166,7 @@ static cudaError_t launch_sk(const SketchArgs &a, cudaStream_t st)
     const int64_t grid = tiles < cap ? tiles : cap;
     kern<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(
         static_cast<const uint8_t *>(a.x), a.nvec, a.m, static_cast<const uint16_t *>(a.proj), a.signs, a.norms);
+    note_launch("sketch_kernel");
     return cudaGetLastError();
 }
 
@@ -207,6 +193,7 @@ static cudaError_t launch_q5(const QuantArgs &a, cudaStream_t st)
         const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
         kern<<<(unsigned)(grid > 0 ? grid : 1), kW5 * 32, smem, st>>>(a.tmap_v32, a.nblocks, *a.tables,
                                                                      static_cast<uint8_t *>(a.codes), a.norms);
+        note_launch("quantize_v5_kernel");
         return cudaGetLastError();
     }
 }
@@ -231,6 +218,7 @@ static cudaError_t launch_dq5(const DequantArgs &a, cudaStream_t st)
                 const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
                 kp<<<(unsigned)(grid > 0 ? grid : 1), kW5 * 32, smemp, st>>>(
                     static_cast<const uint8_t *>(a.codes), a.norms, a.nblocks, *a.tables, a.tmap_out32);
+                note_launch("dequantize_v5p_kernel");
                 return cudaGetLastError();
             }
         }
@@ -244,6 +232,7 @@ static cudaError_t launch_dq5(const DequantArgs &a, cudaStream_t st)
         const int64_t grid = want < (int64_t)a.num_sms ? want : (int64_t)a.num_sms;
         kern<<<(unsigned)(grid > 0 ? grid : 1), kW5 * 32, smem, st>>>(static_cast<const uint8_t *>(a.codes),
                                                                      a.norms, a.nblocks, *a.tables, a.tmap_out32);
+        note_launch("dequantize_v5_kernel");
         return cudaGetLastError();
     }
 }
@@ -268,6 +257,7 @@ static cudaError_t launch_qjl8(const QuantArgs &a, cudaStream_t st)
         kern<<<(unsigned)(grid > 0 ? grid : 1), kW8 * 32, smem, st>>>(
             a.tmap_v, a.tmap_s, a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms, a.m, a.qsigns,
             a.qnorms);
+        note_launch("qjl_v8_quant_kernel");
         return cudaGetLastError();
     }
 }
@@ -292,6 +282,7 @@ static cudaError_t launch_qjl7(const QuantArgs &a, cudaStream_t st)
         kern<<<(unsigned)(grid > 0 ? grid : 1), kW7 * 32, smem, st>>>(
             a.tmap_v, a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms, a.m,
             a.tmap_s, a.qsigns, a.qnorms);
+        note_launch("qjl_v7_quant_kernel");
         return cudaGetLastError();
     }
 }
@@ -317,6 +308,7 @@ static cudaError_t launch_qjl6(const QuantArgs &a, cudaStream_t st)
         kern<<<(unsigned)(grid > 0 ? grid : 1), kW6 * 32, smem, st>>>(
             a.tmap_v, a.nblocks, *a.tables, static_cast<uint8_t *>(a.codes), a.norms, a.m,
             a.tmap_s, a.qsigns, a.qnorms);
+        note_launch("qjl_v6_quant_kernel");
         return cudaGetLastError();
     }
 }
@@ -382,8 +374,6 @@ cudaError_t RQ_CAT(launch_sketch, RQ_D, RQ_DT)(const SketchArgs &a, cudaStream_t
     if (RQ_D == 128) {
         cudaError_t e3 = launch_sketch_v3<RQ_BF16>(a, st);
         if (e3 != cudaErrorNotSupported) return e3;
-        cudaError_t e2 = launch_sketch_v2<RQ_BF16>(a, st);
-        if (e2 != cudaErrorNotSupported) return e2;
     }
     QuantTables T{};
     cudaError_t e = launch_mma<RQ_D, 1, RQ_BF16, 1>(T, a.x, a.nvec, nullptr, nullptr, a.m, a.proj, a.signs, a.norms,

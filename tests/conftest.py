@@ -30,3 +30,9 @@ def cuda_dev():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_sessionfinish(session, exitstatus):
+    mod = sys.modules.get("tests.gpu_checks") or sys.modules.get("gpu_checks")
+    if mod is not None:
+        mod.write_report()

@@ -1,22 +1,9 @@
-"""GPU parity: librq (through its C ABI) against the CPU oracle.
-
-Bars (from the arithmetic each side follows):
-  * codes, norms, reconstructions, residual norms, the projection matrix:
-    bit-exact (both sides compute in the same canonical fp32 order); any code
-    mismatch must also sit within 1e-5 of a decision boundary and their count
-    stay below 1e-6 of the elements;
-  * sign bits: bit-exact except where |P_i| / ||v|| <= 1e-5 (the GPU
-    accumulates in fp32, the oracle in fp64), count below 1e-6 of the bits
-    (at these sizes: zero);
-  * scores: |gpu - oracle| <= 1e-3 * ||q|| * (n16 + rn16) -- the error scale
-    of a dot product of that size (the oracle is fp64 from the same inputs;
-    the GPU rounds intermediates to fp32).
-Inputs are the seeded recipes of kv_quantization_b200.synth at sizes the
-oracle finishes in seconds, spanning several tiles with a ragged tail, plus
-sampled checks at the full workload sizes.
+"""GPU parity: librq (through its C ABI) against the CPU oracle, on inputs
+the oracle finishes in seconds that still span several tiles with a ragged
+tail (the bars are listed in tests/gpu_checks.py).  Every case also names the
+kernel the dispatch must have chosen for it (rq_last_launch), so that each
+kernel the library can launch is compared with the oracle somewhere.
 """
-import math
-
 import numpy as np
 import pytest
 import torch
@@ -24,10 +11,9 @@ import torch
 import oracle as O
 from kv_quantization_b200 import _lib as L
 from kv_quantization_b200 import synth
+from tests.gpu_checks import (DEV, check_codes, check_scores, check_signs, dt_code, score_tol, u16)
 
 pytestmark = pytest.mark.gpu
-
-DEV = "cuda:0"
 
 
 @pytest.fixture(autouse=True)
@@ -38,47 +24,12 @@ def no_device_timeouts():
     assert L.rq_device_error(True) == 0
 
 
-def u16(t):
-    return synth.as_u16(t).reshape(-1)
-
-
-def dt_code(dtype):
-    return O.BF16 if dtype == torch.bfloat16 else O.F16
-
-
 def run_quant(x, d, bits, layout, use_signs, seed, cent):
     n = x.numel()
     codes = torch.empty(L.rq_code_bytes(n, d, bits, layout), dtype=torch.uint8, device=DEV)
     norms = torch.empty(n // d, dtype=torch.int16, device=DEV)
     L.rq_quantize(x, d, bits, layout, use_signs, seed, cent, codes, norms)
     return codes, norms
-
-
-def check_codes(g_codes, o_codes, x16, dtype, d, bits, layout, signs, cent):
-    """Bit-exact codes, or mismatches confined to the 1e-5 boundary window."""
-    if np.array_equal(g_codes, o_codes):
-        return 0
-    nb = x16.size // d
-    gi = O.unpack_codes(g_codes, nb, d, bits, layout)
-    oi = O.unpack_codes(o_codes, nb, d, bits, layout)
-    bad = np.nonzero(gi != oi)[0]
-    y64 = O.rotate_f64(x16, dtype, d, signs)
-    t = O.boundaries(cent).astype(np.float64)
-    near = np.min(np.abs(y64[bad][:, None] - t[None, :]), axis=1) <= 1e-5
-    assert near.all(), f"{(~near).sum()} code mismatches outside the boundary window"
-    assert bad.size < 1e-6 * x16.size, f"{bad.size} windowed mismatches"
-    return bad.size
-
-
-def check_signs(g, o, p_rel, n, m):
-    if np.array_equal(g, o):
-        return 0
-    gb = np.unpackbits(g.reshape(n, m // 8), axis=1, bitorder="little")
-    ob = np.unpackbits(o.reshape(n, m // 8), axis=1, bitorder="little")
-    bad = np.nonzero((gb != ob).reshape(-1))[0]
-    assert np.all(np.abs(p_rel[bad]) <= 1e-5), "sign mismatch outside the window"
-    assert bad.size < max(1.0, 1e-6 * n * m), f"{bad.size} windowed sign mismatches"
-    return bad.size
 
 
 # ------------------------------------------------------------------ quantize / dequantize
@@ -99,6 +50,21 @@ def test_fp16_int8_256x512_full():
     assert np.array_equal(u16(out), oo)
 
 
+def quant_kernels(d, bits, layout):
+    """Kernels the dispatch picks for rq_quantize / rq_dequantize: the d = 128
+    one-block-per-thread kernels when a saturating search grid exists (1-6
+    bits), the general-d kernels otherwise; 1-3-bit packed d = 128 codes take
+    the pair-table dequantize."""
+    q = "quantize_v5_kernel" if d == 128 and bits <= 6 else "quantize_v2_kernel"
+    if d != 128:
+        dq = "dequantize_v2_kernel"
+    elif layout == L.RQ_CODES_PACKED and bits <= 3:
+        dq = "dequantize_v5p_kernel"
+    else:
+        dq = "dequantize_v5_kernel"
+    return q, dq
+
+
 CASES = [
     # d, bits, layout, dtype, signs
     (128, 4, L.RQ_CODES_PACKED, torch.bfloat16, 1),
@@ -107,6 +73,7 @@ CASES = [
     (128, 2, L.RQ_CODES_PACKED, torch.float16, 0),
     (128, 1, L.RQ_CODES_PACKED, torch.bfloat16, 1),
     (128, 8, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    (128, 7, L.RQ_CODES_INT8, torch.float16, 1),
     (128, 4, L.RQ_CODES_INT8, torch.float16, 1),
     (128, 6, L.RQ_CODES_PACKED, torch.bfloat16, 0),
     (64, 4, L.RQ_CODES_PACKED, torch.bfloat16, 1),
@@ -123,9 +90,12 @@ def test_quant_dequant_parity(d, bits, layout, dtype, signs):
     nblocks = 3 * 128 + 7                                     # several tiles, ragged tail
     x = synth.student_t_outliers(1, nblocks * d, seed=100 + d + bits, dtype=dtype, device=DEV).reshape(-1)
     cent = L.rq_lloyd_max(bits)
+    kq, kdq = quant_kernels(d, bits, layout)
     codes, norms = run_quant(x, d, bits, layout, signs, 1234 + bits, cent)
+    assert L.rq_last_launch() == kq
     out = torch.empty_like(x)
     L.rq_dequantize(codes, norms, x.numel(), d, bits, layout, signs, 1234 + bits, cent, out)
+    assert L.rq_last_launch() == kdq
     torch.cuda.synchronize()
     x16 = u16(x)
     s = O.sign_diagonal(1234 + bits, d) if signs else None
@@ -157,6 +127,7 @@ def test_binary_search_fallback_table():
     cent[8] = cent[7] + 1e-6
     x = synth.gaussian_matrix(64, 1024, 1.0, seed=5, dtype=torch.bfloat16, device=DEV)
     codes, norms = run_quant(x, 128, 4, L.RQ_CODES_PACKED, 1, 9, cent)
+    assert L.rq_last_launch() == "quantize_v2_kernel"
     torch.cuda.synchronize()
     x16 = u16(x)
     oc, on, _, _ = O.quantize(x16, O.BF16, 128, 4, O.PACKED, O.sign_diagonal(9, 128), cent)
@@ -249,12 +220,30 @@ def test_llama7b_32_layers_one_call_sampled():
 def test_projection_bit_exact(m, d, dtype):
     S = torch.empty(m, d, dtype=dtype, device=DEV)
     L.qjl_make_projection(77 + m, m, d, S)
+    assert L.rq_last_launch() == "projection_kernel"
     torch.cuda.synchronize()
     assert np.array_equal(u16(S), O.projection(77 + m, m, d, dt_code(dtype)).reshape(-1))
 
 
-@pytest.mark.parametrize("d,m", [(128, 256), (128, 128), (256, 256), (512, 512), (64, 40)])
-def test_sketch_keys(d, m):
+# Key sketch: d = 128 with m <= 256 takes the warp-specialised TMA kernel; the
+# tensor-core fallback covers the shapes whose S and tile fit in shared memory;
+# the CUDA-core kernel the rest.
+SKETCH_CASES = [
+    # d, m, kernel
+    (128, 256, "sketch_v3_kernel"),
+    (128, 128, "sketch_v3_kernel"),
+    (128, 72, "sketch_v3_kernel"),
+    (128, 512, "qjl_mma_kernel<sketch>"),
+    (256, 256, "qjl_mma_kernel<sketch>"),
+    (256, 264, "sketch_kernel"),
+    (512, 32, "qjl_mma_kernel<sketch>"),
+    (512, 512, "sketch_kernel"),
+    (64, 40, "qjl_mma_kernel<sketch>"),
+]
+
+
+@pytest.mark.parametrize("d,m,kernel", SKETCH_CASES)
+def test_sketch_keys(d, m, kernel):
     n = 2 * 301
     k = synth.kv_with_channels(1, 2, 301, d, seed=3, device=DEV).reshape(-1)
     S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
@@ -262,6 +251,7 @@ def test_sketch_keys(d, m):
     signs = torch.empty(n * m // 8, dtype=torch.uint8, device=DEV)
     norms = torch.empty(n, dtype=torch.int16, device=DEV)
     L.qjl_sketch(k, d, m, S, signs, norms)
+    assert L.rq_last_launch() == kernel
     torch.cuda.synchronize()
     k16 = u16(k)
     os_, p = O.sketch(k16, O.BF16, d, m, u16(S), want_p=True)
@@ -269,59 +259,90 @@ def test_sketch_keys(d, m):
     assert np.array_equal(norms.cpu().numpy().view(np.uint16), O.vec_norms(k16, O.BF16, d))
 
 
+# Fused quantize + residual sketch: one kernel per head dim when a saturating
+# search grid exists (bits <= 6) and S's tiles fit; then the pipelined
+# fallback for d = 128 / 256 (7-8-bit tables); then the unpipelined
+# tensor-core kernel (any d whose S fits in shared memory); then CUDA cores.
 QJL_CASES = [
-    # d, bits, m, layout, dtype, signs
-    (128, 4, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1),
-    (128, 3, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1),
-    (128, 5, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1),
-    (128, 1, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1),
-    (128, 2, 40, L.RQ_CODES_PACKED, torch.float16, 0),
-    (128, 6, 64, L.RQ_CODES_INT8, torch.float16, 1),
-    (256, 2, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1),
-    (256, 4, 72, L.RQ_CODES_PACKED, torch.float16, 1),
-    (256, 3, 128, L.RQ_CODES_INT8, torch.bfloat16, 0),
-    (512, 2, 512, L.RQ_CODES_PACKED, torch.bfloat16, 1),
-    (512, 3, 72, L.RQ_CODES_PACKED, torch.float16, 0),
-    (512, 4, 264, L.RQ_CODES_PACKED, torch.bfloat16, 1),
+    # d, bits, m, layout, dtype, signs, kernel
+    (128, 4, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v6_quant_kernel"),
+    (128, 3, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v6_quant_kernel"),
+    (128, 5, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v6_quant_kernel"),
+    (128, 1, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v6_quant_kernel"),
+    (128, 2, 40, L.RQ_CODES_PACKED, torch.float16, 0, "qjl_v6_quant_kernel"),
+    (128, 6, 64, L.RQ_CODES_INT8, torch.float16, 1, "qjl_v6_quant_kernel"),
+    (256, 2, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v7_quant_kernel"),
+    (256, 4, 72, L.RQ_CODES_PACKED, torch.float16, 1, "qjl_v7_quant_kernel"),
+    (256, 3, 128, L.RQ_CODES_INT8, torch.bfloat16, 0, "qjl_v7_quant_kernel"),
+    (512, 2, 512, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v8_quant_kernel"),
+    (512, 3, 72, L.RQ_CODES_PACKED, torch.float16, 0, "qjl_v8_quant_kernel"),
+    (128, 7, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v3_quant_kernel"),
+    (128, 8, 256, L.RQ_CODES_INT8, torch.float16, 0, "qjl_v3_quant_kernel"),
+    (256, 8, 64, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v3_quant_kernel"),
+    (64, 3, 72, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_mma_kernel<fused>"),
+    (64, 8, 128, L.RQ_CODES_INT8, torch.float16, 1, "qjl_mma_kernel<fused>"),
+    (128, 4, 264, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_mma_kernel<fused>"),
+    (512, 8, 16, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_mma_kernel<fused>"),
+    (512, 4, 264, L.RQ_CODES_PACKED, torch.bfloat16, 1, "quantize_kernel"),
+    (256, 2, 512, L.RQ_CODES_PACKED, torch.float16, 1, "quantize_kernel"),
 ]
 
 
-@pytest.mark.parametrize("d,bits,m,layout,dtype,signs", QJL_CASES)
-def test_quantize_qjl_residual(d, bits, m, layout, dtype, signs):
+def run_fused(x, d, bits, layout, signs, seed, cent, m, S):
+    nblocks = x.numel() // d
+    codes = torch.empty(L.rq_code_bytes(x.numel(), d, bits, layout), dtype=torch.uint8, device=DEV)
+    norms = torch.empty(nblocks, dtype=torch.int16, device=DEV)
+    qs = torch.empty(nblocks * m // 8, dtype=torch.uint8, device=DEV)
+    qn = torch.empty(nblocks, dtype=torch.int16, device=DEV)
+    L.rq_quantize_qjl(x, d, bits, layout, signs, seed, cent, m, S, codes, norms, qs, qn)
+    return codes, norms, qs, qn
+
+
+def check_fused(x16, dt, d, bits, layout, signs, seed, cent, m, S16, codes, norms, qs, qn, full_blocks=None):
+    """Codes, norms, residual norms bit-exact; residual sign bits windowed."""
+    nb = x16.size // d
+    s = O.sign_diagonal(seed, d) if signs else None
+    oc, on, _, _ = O.quantize(x16, dt, d, bits, layout, s, cent)
+    check_codes(codes, oc, x16, dt, d, bits, layout, s, cent)
+    assert np.array_equal(norms, on)
+    r_bf, rn = O.residual(x16, dt, oc, on, d, bits, layout, s, cent)
+    assert np.array_equal(qn, rn)
+    osg, p = O.sketch(r_bf, O.BF16, d, m, S16, want_p=True)
+    check_signs(qs, osg, p, nb, m, full_bits=None if full_blocks is None else full_blocks * m)
+
+
+@pytest.mark.parametrize("d,bits,m,layout,dtype,signs,kernel", QJL_CASES)
+def test_quantize_qjl_residual(d, bits, m, layout, dtype, signs, kernel):
     nblocks = 2 * 128 + 11
     x = synth.student_t_outliers(1, nblocks * d, seed=7 + d + m, dtype=dtype, device=DEV).reshape(-1)
     cent = L.rq_lloyd_max(bits)
     S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
     L.qjl_make_projection(2, m, d, S)
-    codes = torch.empty(L.rq_code_bytes(x.numel(), d, bits, layout), dtype=torch.uint8, device=DEV)
-    norms = torch.empty(nblocks, dtype=torch.int16, device=DEV)
-    qs = torch.empty(nblocks * m // 8, dtype=torch.uint8, device=DEV)
-    qn = torch.empty(nblocks, dtype=torch.int16, device=DEV)
-    L.rq_quantize_qjl(x, d, bits, layout, signs, 1, cent, m, S, codes, norms, qs, qn)
+    codes, norms, qs, qn = run_fused(x, d, bits, layout, signs, 1, cent, m, S)
+    assert L.rq_last_launch() == kernel
     torch.cuda.synchronize()
-    x16 = u16(x)
-    dt = dt_code(dtype)
-    s = O.sign_diagonal(1, d) if signs else None
-    oc, on, _, _ = O.quantize(x16, dt, d, bits, layout, s, cent)
-    check_codes(codes.cpu().numpy(), oc, x16, dt, d, bits, layout, s, cent)
-    assert np.array_equal(norms.cpu().numpy().view(np.uint16), on)
-    r_bf, rn = O.residual(x16, dt, oc, on, d, bits, layout, s, cent)
-    assert np.array_equal(qn.cpu().numpy().view(np.uint16), rn)
-    osg, p = O.sketch(r_bf, O.BF16, d, m, u16(S), want_p=True)
-    check_signs(qs.cpu().numpy(), osg, p, nblocks, m)
+    check_fused(u16(x), dt_code(dtype), d, bits, layout, signs, 1, cent, m, u16(S), codes.cpu().numpy(),
+                norms.cpu().numpy().view(np.uint16), qs.cpu().numpy(), qn.cpu().numpy().view(np.uint16))
 
 
-def _score_tol(q16, G, nq, d, sk_norms, norms=None):
-    qf = (q16.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(G, nq, d)
-    qn = np.linalg.norm(qf, axis=2)[:, :, None]
-    kn = np.array([O.f16_to_f32(int(h)) for h in sk_norms.reshape(-1)]).reshape(G, 1, -1)
-    if norms is not None:
-        kn = kn + np.array([O.f16_to_f32(int(h)) for h in norms.reshape(-1)]).reshape(G, 1, -1)
-    return 1e-3 * qn * kn
+# ------------------------------------------------------------------ scores
+
+def make_two_stage(G, T, d, bits, m, layout, seed, sseed, pseed):
+    k = synth.normal((G, T, d), seed=seed, device=DEV).reshape(-1)
+    cent = L.rq_lloyd_max(bits)
+    S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
+    L.qjl_make_projection(pseed, m, d, S)
+    codes, norms, qs, qn = run_fused(k, d, bits, layout, 1, sseed, cent, m, S)
+    return k, cent, S, codes, norms, qs, qn
 
 
-def test_score_pure_qjl():
-    G, nq, T, d, m = 3, 32, 333, 128, 256
+def score_kernels(nq):
+    return "score_v2_prologue,score_v4_kernel" if nq <= 128 else "score_prologue_kernel,score_kernel"
+
+
+@pytest.mark.parametrize("nq", [32, 160])
+def test_score_pure_qjl(nq):
+    G, T, d, m = 3, 333, 128, 256
     k = synth.kv_with_channels(1, G, T, d, seed=4, device=DEV).reshape(-1)
     q = synth.normal((G, nq, d), seed=5, device=DEV)
     S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
@@ -332,11 +353,12 @@ def test_score_pure_qjl():
     scores = torch.empty(G, nq, T, dtype=torch.float32, device=DEV)
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, signs, kn, T, scores, ws)
+    assert L.rq_last_launch() == score_kernels(nq)
     torch.cuda.synchronize()
     q16 = u16(q)
-    want = O.score(q16, G, nq, d, m, u16(S), O.BF16, signs.cpu().numpy(), kn.cpu().numpy().view(np.uint16), T)
-    err = np.abs(scores.cpu().numpy().astype(np.float64) - want)
-    assert np.all(err <= _score_tol(q16, G, nq, d, kn.cpu().numpy().view(np.uint16)))
+    kn16 = kn.cpu().numpy().view(np.uint16)
+    want = O.score(q16, G, nq, d, m, u16(S), O.BF16, signs.cpu().numpy(), kn16, T)
+    check_scores(scores.cpu().numpy(), want, score_tol(q16, G, nq, d, kn16), f"pure d={d} m={m} nq={nq}")
 
 
 def test_score_fp16_projection_ragged_queries():
@@ -357,65 +379,50 @@ def test_score_fp16_projection_ragged_queries():
     L.qjl_score(q, G, nq, d, m, S16, signs, kn, T, scores, ws)
     torch.cuda.synchronize()
     q16 = u16(q)
-    want = O.score(q16, G, nq, d, m, u16(S16), O.F16, signs.cpu().numpy(), kn.cpu().numpy().view(np.uint16), T)
-    err = np.abs(scores.cpu().numpy().astype(np.float64) - want)
-    assert np.all(err <= _score_tol(q16, G, nq, d, kn.cpu().numpy().view(np.uint16)))
+    kn16 = kn.cpu().numpy().view(np.uint16)
+    want = O.score(q16, G, nq, d, m, u16(S16), O.F16, signs.cpu().numpy(), kn16, T)
+    check_scores(scores.cpu().numpy(), want, score_tol(q16, G, nq, d, kn16), "pure fp16 S nq=33")
 
 
 @pytest.mark.parametrize("d", [256, 512])
 def test_score_two_stage(d):
     """2-bit rotated Lloyd-Max keys + QJL (m = d) residual sketch, 32 queries."""
     G, nq, T, m, bits = 2, 32, 257, d, 2
-    k = synth.normal((G, T, d), seed=6, device=DEV).reshape(-1)
+    k, cent, S, codes, norms, qs, qn = make_two_stage(G, T, d, bits, m, L.RQ_CODES_PACKED, 6, 4, 5)
     q = synth.normal((G, nq, d), seed=7, device=DEV)
-    cent = L.rq_lloyd_max(bits)
-    S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
-    L.qjl_make_projection(5, m, d, S)
-    codes = torch.empty(L.rq_code_bytes(k.numel(), d, bits, L.RQ_CODES_PACKED), dtype=torch.uint8, device=DEV)
-    norms = torch.empty(G * T, dtype=torch.int16, device=DEV)
-    qs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=DEV)
-    qn = torch.empty(G * T, dtype=torch.int16, device=DEV)
-    L.rq_quantize_qjl(k, d, bits, L.RQ_CODES_PACKED, 1, 4, cent, m, S, codes, norms, qs, qn)
     scores = torch.empty(G, nq, T, dtype=torch.float32, device=DEV)
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits,
                 layout=L.RQ_CODES_PACKED, use_signs=1, sign_seed=4, centroids=cent)
+    assert L.rq_last_launch() == score_kernels(nq)
     torch.cuda.synchronize()
     q16 = u16(q)
-    s = O.sign_diagonal(4, d)
+    n16 = norms.cpu().numpy().view(np.uint16)
     want = O.score(q16, G, nq, d, m, u16(S), O.BF16, qs.cpu().numpy(), qn.cpu().numpy().view(np.uint16), T,
-                   codes=codes.cpu().numpy(), norms=norms.cpu().numpy().view(np.uint16), bits=bits,
-                   layout=O.PACKED, signs_diag=s, c32=cent)
-    err = np.abs(scores.cpu().numpy().astype(np.float64) - want)
-    tol = _score_tol(q16, G, nq, d, qn.cpu().numpy().view(np.uint16), norms.cpu().numpy().view(np.uint16))
-    assert np.all(err <= tol), float((err / tol).max())
+                   codes=codes.cpu().numpy(), norms=n16, bits=bits, layout=O.PACKED,
+                   signs_diag=O.sign_diagonal(4, d), c32=cent)
+    check_scores(scores.cpu().numpy(), want, score_tol(q16, G, nq, d, n16), f"two-stage d={d}")
 
 
 @pytest.mark.parametrize("d,bits,m,nq,layout", [(128, 4, 128, 40, L.RQ_CODES_INT8), (64, 3, 72, 7, L.RQ_CODES_PACKED),
-                                                 (128, 5, 256, 33, L.RQ_CODES_PACKED)])
+                                                 (128, 5, 256, 33, L.RQ_CODES_PACKED),
+                                                 (128, 4, 128, 136, L.RQ_CODES_PACKED),
+                                                 (256, 2, 256, 129, L.RQ_CODES_PACKED)])
 def test_score_two_stage_shapes(d, bits, m, nq, layout):
-    """Query counts that are not multiples of 32, m not a multiple of 64,
-    int8 codes, and a ragged token tail."""
+    """Query counts that are not multiples of 32 (and above 128: the CUDA-core
+    score), m not a multiple of 64, int8 codes, and a ragged token tail."""
     G, T = 3, 131
-    k = synth.normal((G, T, d), seed=16, device=DEV).reshape(-1)
+    k, cent, S, codes, norms, qs, qn = make_two_stage(G, T, d, bits, m, layout, 16, 9, 8)
     q = synth.normal((G, nq, d), seed=17, device=DEV)
-    cent = L.rq_lloyd_max(bits)
-    S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
-    L.qjl_make_projection(8, m, d, S)
-    codes = torch.empty(L.rq_code_bytes(k.numel(), d, bits, layout), dtype=torch.uint8, device=DEV)
-    norms = torch.empty(G * T, dtype=torch.int16, device=DEV)
-    qs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=DEV)
-    qn = torch.empty(G * T, dtype=torch.int16, device=DEV)
-    L.rq_quantize_qjl(k, d, bits, layout, 1, 9, cent, m, S, codes, norms, qs, qn)
     scores = torch.empty(G, nq, T, dtype=torch.float32, device=DEV)
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4 + 1, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits, layout=layout,
                 use_signs=1, sign_seed=9, centroids=cent)
+    assert L.rq_last_launch() == score_kernels(nq)
     torch.cuda.synchronize()
     q16 = u16(q)
+    n16 = norms.cpu().numpy().view(np.uint16)
     want = O.score(q16, G, nq, d, m, u16(S), O.BF16, qs.cpu().numpy(), qn.cpu().numpy().view(np.uint16), T,
-                   codes=codes.cpu().numpy(), norms=norms.cpu().numpy().view(np.uint16), bits=bits,
-                   layout=layout, signs_diag=O.sign_diagonal(9, d), c32=cent)
-    err = np.abs(scores.cpu().numpy().astype(np.float64) - want)
-    tol = _score_tol(q16, G, nq, d, qn.cpu().numpy().view(np.uint16), norms.cpu().numpy().view(np.uint16))
-    assert np.all(err <= tol), float((err / tol).max())
+                   codes=codes.cpu().numpy(), norms=n16, bits=bits, layout=layout,
+                   signs_diag=O.sign_diagonal(9, d), c32=cent)
+    check_scores(scores.cpu().numpy(), want, score_tol(q16, G, nq, d, n16), f"two-stage d={d} b={bits} nq={nq}")

@@ -142,3 +142,13 @@ def test_table_cache_miss_and_hit_paths():
         with pytest.raises(L.RQError) as e:
             _q(FakeTensor(0x30000), bits=bits)
         assert e.value.status == -5
+
+
+def test_probe_and_trace_validate_before_any_launch():
+    """rq_probe_bounded_wait rejects a poll limit out of range without a GPU;
+    a call that fails validation leaves the launch trace empty."""
+    for polls in (0, (1 << 20) + 1):
+        assert L.lib().rq_probe_bounded_wait(polls, None) == -1
+        assert L.rq_last_launch() == ""
+    assert L.lib().rq_quantize(None, 1, 128, 96, 4, 0, 0, 0, None, None, None, None) == -1
+    assert L.rq_last_launch() == ""
