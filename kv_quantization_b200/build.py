@@ -4,8 +4,9 @@
 
 Each .cu under csrc/ compiles to an object in parallel (nvcc -gencode
 arch=compute_100a,code=sm_100a -lineinfo -O3, position-independent), then the
-objects link into kv_quantization_b200/librq.so.  No fast-math: the kernels
-rely on IEEE-rounded fp32 adds, multiplies, reciprocals and square roots.
+objects link into kv_quantization_b200/librq.so.  No fast-math and no
+multiply-add contraction: the kernels rely on IEEE-rounded fp32 adds,
+multiplies, reciprocals and square roots, each rounded on its own.
 """
 from __future__ import annotations
 
@@ -25,8 +26,12 @@ OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "librq.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# --fmad=false: no multiply-add contraction anywhere.  The canonical arithmetic
+# rounds every product and every sum separately; the packed f32x2 intrinsics
+# were measured to be contracted otherwise (the residual x - w * s came out
+# with a single rounding).  Explicit fma intrinsics are unaffected.
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-rdc=true", "-Xcompiler", "-fPIC", "-Xcompiler", "-fno-fast-math",
-              "--ftz=false", "--prec-div=true", "--prec-sqrt=true", "-I", INCLUDE, "-I", CSRC]
+              "--ftz=false", "--prec-div=true", "--prec-sqrt=true", "--fmad=false", "-I", INCLUDE, "-I", CSRC]
 
 
 def nvcc() -> str:

@@ -39,6 +39,17 @@ __device__ __forceinline__ void unpack2(uint32_t w, float &a, float &b)
     }
 }
 
+// x - p * s with the product and the difference each rounded to nearest
+// (the canonical two roundings), written as a packed multiply feeding an FMA
+// with factor -1.  ptxas (CUDA 12.9, sm_100a) was measured to contract a
+// packed f32x2 multiply feeding a packed f32x2 add -- and an FMA with factor
+// +1 -- into one fused multiply-add, even with explicit .rn and
+// --fmad=false; this form was measured to keep both roundings.
+__device__ __forceinline__ float2 sub_mul2_rn(float2 x, float2 p, float2 s)
+{
+    return __ffma2_rn(__fmul2_rn(p, s), make_float2(-1.0f, -1.0f), x);
+}
+
 // Two fp32 -> packed 16-bit pair, round to nearest even.
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float a, float b)

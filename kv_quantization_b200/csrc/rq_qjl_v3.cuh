@@ -183,14 +183,14 @@ qjl_v3_quant_kernel(const __grid_constant__ CUtensorMap tmv, int64_t nblocks, co
                 P[i2].y = cent_lane[unpack_code<kE2, PW>(w, i2 + 32) * 32];
             }
             fwht_row<TPB>(P, part);
-            const float nsc = -__fmul_rn(h16_to_f32(n16), 1.0f / (float)D);
-            const float2 nsc2 = make_float2(nsc, nsc);
+            const float sc = __fmul_rn(h16_to_f32(n16), 1.0f / (float)D);
+            const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
             for (int i2 = 0; i2 < 32; ++i2) {
                 float2 x;
                 x.x = half_of<BF16>(u[i2 >> 1], i2 & 1);
                 x.y = half_of<BF16>(u[16 + (i2 >> 1)], i2 & 1);
-                P[i2] = __fadd2_rn(x, __fmul2_rn(P[i2], nsc2));
+                P[i2] = sub_mul2_rn(x, P[i2], sc2);
             }
             const float rn32 = __fsqrt_rn(combine_parts<TPB>(row_sumsq(P)));
             if (valid && part == 0) qnorms[gblk] = norm_to_h16(rn32);

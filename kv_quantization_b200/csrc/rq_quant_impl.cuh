@@ -119,9 +119,10 @@ __device__ __forceinline__ float block_norm(const float *v)
 }
 
 
-// Sign bits of S v for one vector held as TPB parts of E values: P_i in fp32
-// (FMA accumulation; the bit is exact except when |P_i| is within rounding of
-// zero), bit i = (P_i >= 0), stored LSB-first, 8 per byte, when dst != nullptr.
+// Sign bits of S v for one vector held as TPB parts of E values (each value
+// a 16-bit number widened to fp32): P_i accumulated in fp64 from exact
+// products, so the bit is the sign of the exact dot product; bit i =
+// (P_i >= 0), stored LSB-first, 8 per byte, when dst != nullptr.
 template <int E, int TPB, bool SBF16>
 __device__ __forceinline__ void sketch_signs(const float *v, const void *proj, int D, int m, int part, uint8_t *dst)
 {
@@ -130,18 +131,22 @@ __device__ __forceinline__ void sketch_signs(const float *v, const void *proj, i
     uint32_t word = 0u;
     for (int i = 0; i < m; ++i) {
         const uint4 *Si = reinterpret_cast<const uint4 *>(Sb + (size_t)i * D * 2);
-        float acc = 0.0f;
+        double acc = 0.0;
 #pragma unroll
         for (int k = 0; k < NCH; ++k) {
-            uint4 s = __ldg(Si + k);
-            float a0, a1;
-            unpack2<SBF16>(s.x, a0, a1); acc = __fmaf_rn(a0, v[8 * k + 0], acc); acc = __fmaf_rn(a1, v[8 * k + 1], acc);
-            unpack2<SBF16>(s.y, a0, a1); acc = __fmaf_rn(a0, v[8 * k + 2], acc); acc = __fmaf_rn(a1, v[8 * k + 3], acc);
-            unpack2<SBF16>(s.z, a0, a1); acc = __fmaf_rn(a0, v[8 * k + 4], acc); acc = __fmaf_rn(a1, v[8 * k + 5], acc);
-            unpack2<SBF16>(s.w, a0, a1); acc = __fmaf_rn(a0, v[8 * k + 6], acc); acc = __fmaf_rn(a1, v[8 * k + 7], acc);
+            const uint4 s = __ldg(Si + k);
+            const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float a0, a1;
+                unpack2<SBF16>(sw[q], a0, a1);
+                acc = fma((double)a0, (double)v[8 * k + 2 * q], acc);
+                acc = fma((double)a1, (double)v[8 * k + 2 * q + 1], acc);
+            }
         }
-        acc = combine_parts<TPB>(acc);
-        word |= (acc >= 0.0f ? 1u : 0u) << (i & 7);
+#pragma unroll
+        for (int off = 1; off < TPB; off *= 2) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        word |= (acc >= 0.0 ? 1u : 0u) << (i & 7);
         if ((i & 7) == 7) {
             if (dst) dst[i >> 3] = (uint8_t)word;
             word = 0u;
@@ -224,7 +229,7 @@ quantize_kernel(const uint8_t *__restrict__ x, int64_t nblocks, const __grid_con
                 v[j] = __fsub_rn(xr[j], xh);
             }
             const float rn32 = block_norm<E, TPB>(v);
-            // Sketch of bf16(r): P_i = sum_j S_ij r_j (fp32 accumulation).
+            // Sketch of bf16(r): P_i = sum_j S_ij r_j (fp64 accumulation of exact products).
 #pragma unroll
             for (int j = 0; j < E; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
             const int64_t blk = row / TPB;

@@ -82,9 +82,9 @@ __device__ __forceinline__ void load_half64(uint32_t row_base, int blk, uint32_t
     }
 }
 
-// P <- x + P * nsc for the lane's half of the input row.
+// P <- x - P * sc for the lane's half of the input row (two roundings).
 template <bool BF16, bool SIGNS>
-__device__ __forceinline__ void residual_half64(uint32_t row_base, int blk, uint32_t pmask_half, float2 nsc2,
+__device__ __forceinline__ void residual_half64(uint32_t row_base, int blk, uint32_t pmask_half, float2 sc2,
                                                 float2 *P)
 {
 #pragma unroll
@@ -101,7 +101,7 @@ __device__ __forceinline__ void residual_half64(uint32_t row_base, int blk, uint
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float2 x = make_float2(half_of<BF16>(wa[e >> 1], e & 1), half_of<BF16>(wb[e >> 1], e & 1));
-            P[8 * k + e] = __fadd2_rn(x, __fmul2_rn(P[8 * k + e], nsc2));
+            P[8 * k + e] = sub_mul2_rn(x, P[8 * k + e], sc2);
         }
     }
 }
@@ -362,8 +362,8 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
             else if (tile_of(k - 1 + kNSG6) < t1) load_tile(k - 1 + kNSG6);
         }
         fwht_half64(P, hf);
-        const float nsc = -__fmul_rn(h16_to_f32(n16), 1.0f / 128.0f);
-        residual_half64<BF16, SIGNS>(rbase, blk_row, pmh, make_float2(nsc, nsc), P);
+        const float sc = __fmul_rn(h16_to_f32(n16), 1.0f / 128.0f);
+        residual_half64<BF16, SIGNS>(rbase, blk_row, pmh, make_float2(sc, sc), P);
         const float rn32 = __fsqrt_rn(sumsq_half64(P));
         if (valid && hf == 0) qnorms[blk] = norm_to_h16(rn32);
         store_half64<false>(rbase, blk_row, pmh, P);     // r' (signs live in S')

@@ -161,8 +161,8 @@ qjl_v8_quant_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_consta
                 if (q == 0) norms[blk] = n16;
             }
             fwht_half64<8, 4>(P, q);
-            const float nsc = -__fmul_rn(h16_to_f32(n16), 1.0f / 512.0f);
-            residual_half64<BF16, SIGNS>(rbase, blk_row, pmq, make_float2(nsc, nsc), P);
+            const float sc = __fmul_rn(h16_to_f32(n16), 1.0f / 512.0f);
+            residual_half64<BF16, SIGNS>(rbase, blk_row, pmq, make_float2(sc, sc), P);
             const float rn32 = __fsqrt_rn(sumsq_half64<8, 4>(P));
             if (valid && q == 0) qnorms[blk] = norm_to_h16(rn32);
             store_half64<SIGNS>(rbase, blk_row, pmq, P);

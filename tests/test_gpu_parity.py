@@ -52,10 +52,10 @@ def test_fp16_int8_256x512_full():
 
 def quant_kernels(d, bits, layout):
     """Kernels the dispatch picks for rq_quantize / rq_dequantize: the d = 128
-    one-block-per-thread kernels when a saturating search grid exists (1-6
-    bits), the general-d kernels otherwise; 1-3-bit packed d = 128 codes take
-    the pair-table dequantize."""
-    q = "quantize_v5_kernel" if d == 128 and bits <= 6 else "quantize_v2_kernel"
+    one-block-per-thread kernels when a saturating search grid of at most 128
+    cells exists (the Lloyd-Max tables of 1-5 bits), the general-d kernels
+    otherwise; 1-3-bit packed d = 128 codes take the pair-table dequantize."""
+    q = "quantize_v5_kernel" if d == 128 and bits <= 5 else "quantize_v2_kernel"
     if d != 128:
         dq = "dequantize_v2_kernel"
     elif layout == L.RQ_CODES_PACKED and bits <= 3:
@@ -121,10 +121,13 @@ def test_quant_dequant_parity(d, bits, layout, dtype, signs):
 
 
 def test_binary_search_fallback_table():
-    """A table whose thresholds no 128-cell grid separates (two levels 1e-6
-    apart) takes the binary-search path; codes still match exactly."""
+    """A table whose thresholds no 128-cell grid separates (levels 6, 7, 8
+    within 2e-6, so two decision thresholds lie 1e-6 apart) takes the
+    branch-free binary search; codes still match exactly."""
     cent = L.rq_lloyd_max(4).copy()
-    cent[8] = cent[7] + 1e-6
+    cent[7] = cent[6] + 1e-6
+    cent[8] = cent[6] + 2e-6
+    assert np.all(np.diff(cent) > 0)
     x = synth.gaussian_matrix(64, 1024, 1.0, seed=5, dtype=torch.bfloat16, device=DEV)
     codes, norms = run_quant(x, 128, 4, L.RQ_CODES_PACKED, 1, 9, cent)
     assert L.rq_last_launch() == "quantize_v2_kernel"
@@ -260,8 +263,8 @@ def test_sketch_keys(d, m, kernel):
 
 
 # Fused quantize + residual sketch: one kernel per head dim when a saturating
-# search grid exists (bits <= 6) and S's tiles fit; then the pipelined
-# fallback for d = 128 / 256 (7-8-bit tables); then the unpipelined
+# search grid exists (bits <= 5) and S's tiles fit; then the pipelined
+# fallback for d = 128 / 256 (6-8-bit tables); then the unpipelined
 # tensor-core kernel (any d whose S fits in shared memory); then CUDA cores.
 QJL_CASES = [
     # d, bits, m, layout, dtype, signs, kernel
@@ -270,7 +273,8 @@ QJL_CASES = [
     (128, 5, 128, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v6_quant_kernel"),
     (128, 1, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v6_quant_kernel"),
     (128, 2, 40, L.RQ_CODES_PACKED, torch.float16, 0, "qjl_v6_quant_kernel"),
-    (128, 6, 64, L.RQ_CODES_INT8, torch.float16, 1, "qjl_v6_quant_kernel"),
+    (128, 5, 64, L.RQ_CODES_INT8, torch.float16, 1, "qjl_v6_quant_kernel"),
+    (128, 6, 64, L.RQ_CODES_INT8, torch.float16, 1, "qjl_v3_quant_kernel"),
     (256, 2, 256, L.RQ_CODES_PACKED, torch.bfloat16, 1, "qjl_v7_quant_kernel"),
     (256, 4, 72, L.RQ_CODES_PACKED, torch.float16, 1, "qjl_v7_quant_kernel"),
     (256, 3, 128, L.RQ_CODES_INT8, torch.bfloat16, 0, "qjl_v7_quant_kernel"),
