@@ -56,8 +56,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr)
     return v;
 }
 
-// A load the compiler may not merge with an earlier load of the same address
-// (the residual pass re-reads its row instead of keeping it in registers).
+// A shared-memory load the compiler keeps in program order relative to the
+// other volatile asm (the mbarrier waits) and never merges with an earlier
+// load of the same address: every read of smem that a bulk copy or TMA
+// writes asynchronously goes through it, so it cannot be hoisted above the
+// wait that guards the data (the plain lds64 / lds128 above are for tables
+// written before a __syncthreads, or for addresses computed from such data).
 __device__ __forceinline__ uint4 lds128_fresh(uint32_t addr)
 {
     uint4 v;
@@ -127,6 +131,26 @@ __device__ __forceinline__ void put_code(uint32_t *w, int j, uint32_t c)
     if ((b & 31) + PW > 32) w[(b >> 5) + 1] |= c >> (32 - (b & 31));
 }
 
+// put_code of base + (y > t) into zeroed fields: the base is added at its
+// offset (fields never carry into each other, base + 1 < 2^PW when a
+// boundary sits in the cell) and the comparison becomes one predicated add.
+template <int PW>
+__device__ __forceinline__ void put_code_cmp(uint32_t *w, int j, uint32_t base, float y, float t)
+{
+    const int b = j * PW;
+    if ((b & 31) + PW > 32) {
+        put_code<PW>(w, j, base + (y > t ? 1u : 0u));
+    } else {
+        uint32_t v = w[b >> 5] + (base << (b & 31));
+        asm("{\n\t.reg .pred p;\n\t"
+            "setp.gt.f32 p, %1, %2;\n\t"
+            "@p add.u32 %0, %0, %3;\n\t}"
+            : "+r"(v)
+            : "f"(y), "f"(t), "r"(1u << (b & 31)));
+        w[b >> 5] = v;
+    }
+}
+
 // ------------------------------------------------------------------ row of 128
 
 // Row `r` of a chunk/tile whose two 64-value halves are regions `half_bytes`
@@ -137,8 +161,8 @@ __device__ __forceinline__ void load_row128(uint32_t tile, uint32_t half_bytes, 
 {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        uint4 lo = lds128(tile + sw128_offset(r, k));
-        uint4 hi = lds128(tile + half_bytes + sw128_offset(r, k));
+        uint4 lo = lds128_fresh(tile + sw128_offset(r, k));
+        uint4 hi = lds128_fresh(tile + half_bytes + sw128_offset(r, k));
         if constexpr (SIGNS) {
             const uint4 ml = lds128_fresh(pmask_smem + 16u * k);
             const uint4 mh = lds128_fresh(pmask_smem + 128u + 16u * k);
@@ -240,8 +264,8 @@ __device__ __forceinline__ void codes128(const float2 *P, float inv, const SatGr
         uint32_t a0, a1;
         sat_addr(G, y, a0, a1);
         const uint2 e0 = lds64(a0), e1 = lds64(a1);
-        put_code<PW>(w, i, e0.y + (y.x > __uint_as_float(e0.x) ? 1u : 0u));
-        put_code<PW>(w, i + 64, e1.y + (y.y > __uint_as_float(e1.x) ? 1u : 0u));
+        put_code_cmp<PW>(w, i, e0.y, y.x, __uint_as_float(e0.x));
+        put_code_cmp<PW>(w, i + 64, e1.y, y.y, __uint_as_float(e1.x));
     }
 }
 
@@ -288,6 +312,7 @@ quantize_v5_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, con
     uint8_t *wring = ring + (size_t)warp * kNSW5 * kChunkBytes5;
     uint64_t *wfull = full + warp * kNSW5;
     auto issue = [&](int64_t j, int s) {
+        fence_proxy_async_smem();                   // the slot's earlier generic reads precede the copy
         mbar_arrive_expect_tx(&wfull[s], kChunkBytes5);
         uint8_t *dst = wring + (size_t)s * kChunkBytes5;
         tma_load_3d(dst, &tmx, 0, 0, (int)(j * 32), &wfull[s]);
@@ -331,7 +356,7 @@ __host__ __device__ inline int cent_copies5(int levels) { return levels <= 32 ? 
 
 __host__ __device__ inline size_t dequantize_v5_smem(int pw, int levels)
 {
-    return 1024 + (size_t)kW5 * kChunkBytes5 + (size_t)kW5 * kNSD5 * 512 * pw +
+    return 1024 + (size_t)kW5 * kChunkBytes5 + (size_t)kW5 * kNSD5 * (512 * pw + 64) +
            (size_t)levels * cent_copies5(levels) * 4 + 256 + 8 * kW5 * kNSD5;
 }
 
@@ -341,12 +366,13 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
                      const __grid_constant__ QuantTables T, const __grid_constant__ CUtensorMap tmo)
 {
     constexpr int CB = 16 * PW;
-    constexpr uint32_t RING = 512u * PW;          // one chunk's codes
+    constexpr uint32_t RING = 512u * PW;              // one chunk's codes
+    constexpr uint32_t SLOT = RING + 64u;             // ... and its 32 fp16 norms
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *outb = base;                                         // kW5 staging chunks
     uint8_t *cring = outb + (size_t)kW5 * kChunkBytes5;           // kW5 x kNSD5 code chunks
-    float *cent = reinterpret_cast<float *>(cring + (size_t)kW5 * kNSD5 * RING);
+    float *cent = reinterpret_cast<float *>(cring + (size_t)kW5 * kNSD5 * SLOT);
     const int copies = cent_copies5(T.levels);
     uint32_t *pmask = reinterpret_cast<uint32_t *>(cent + T.levels * copies);
     uint64_t *full = reinterpret_cast<uint64_t *>(pmask + 64);
@@ -364,13 +390,22 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
     setup_pair_masks(T, pmask, 128);
     __syncthreads();
 
-    uint8_t *wring = cring + (size_t)warp * kNSD5 * RING;
+    uint8_t *wring = cring + (size_t)warp * kNSD5 * SLOT;
     uint8_t *wout = outb + (size_t)warp * kChunkBytes5;
     uint64_t *wfull = full + warp * kNSD5;
+    // the chunk's codes and the whole 16-byte groups of its norms (the norms
+    // of a ragged last chunk's remaining blocks are read from global memory)
+    auto norm_bytes = [&](int64_t j) -> uint32_t {
+        const int64_t nb = nblocks - j * 32 < 32 ? nblocks - j * 32 : 32;
+        return (uint32_t)(nb * 2) & ~15u;
+    };
     auto issue = [&](int64_t j, int s) {
         const int64_t nb = nblocks - j * 32 < 32 ? nblocks - j * 32 : 32;
-        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(nb * CB));
-        bulk_load(wring + (size_t)s * RING, codes + j * 32 * CB, (uint32_t)(nb * CB), &wfull[s]);
+        const uint32_t nbytes = norm_bytes(j);
+        fence_proxy_async_smem();                   // the slot's earlier generic reads precede the copy
+        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(nb * CB) + nbytes);
+        bulk_load(wring + (size_t)s * SLOT, codes + j * 32 * CB, (uint32_t)(nb * CB), &wfull[s]);
+        if (nbytes) bulk_load(wring + (size_t)s * SLOT + RING, norms + j * 32, nbytes, &wfull[s]);
     };
     if (lane == 0)
         for (int s = 0; s < kNSD5; ++s) {
@@ -384,27 +419,32 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
     // code can address outside the table.
     const uint32_t cmask = PW == 8 ? (uint32_t)T.levels - 1u : 0xffffffffu;
     const uint32_t pm = smem_u32(pmask);
-    auto fetch_norm = [&](int64_t j) -> float {
-        const int64_t blk = j * 32 + lane;
-        return (j < c1 && blk < nblocks) ? h16_to_f32(__ldg(norms + blk)) : 0.0f;
-    };
-    float nrm = fetch_norm(c0 + warp);
 
     for (int64_t k = 0;; ++k) {
         const int64_t j = c0 + warp + k * kW5;
         if (j >= c1) break;
         const int s = (int)(k % kNSD5);
-        const float nrm_next = fetch_norm(j + kW5);
         if (!mbar_wait(&wfull[s], (uint32_t)((k / kNSD5) & 1))) break;
+        float nrm;
+        {
+            const int64_t blk = j * 32 + lane;
+            uint16_t h = 0;
+            if ((uint32_t)lane * 2u < norm_bytes(j)) {
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(h)
+                             : "r"(smem_u32(wring + (size_t)s * SLOT + RING) + (uint32_t)lane * 2u));
+            } else if (blk < nblocks) {
+                h = __ldg(norms + blk);
+            }
+            nrm = h16_to_f32(h);
+        }
         uint32_t cw[4 * PW];
-        const uint32_t src = smem_u32(wring + (size_t)s * RING) + (uint32_t)lane * CB;
+        const uint32_t src = smem_u32(wring + (size_t)s * SLOT) + (uint32_t)lane * CB;
 #pragma unroll
         for (int q = 0; q < PW; ++q) {
-            const uint4 v = lds128(src + 16u * q);
+            const uint4 v = lds128_fresh(src + 16u * q);
             cw[4 * q] = v.x; cw[4 * q + 1] = v.y; cw[4 * q + 2] = v.z; cw[4 * q + 3] = v.w;
         }
-        __syncwarp();
-        if (lane == 0 && j + (int64_t)kNSD5 * kW5 < c1) issue(j + (int64_t)kNSD5 * kW5, s);
         float2 P[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
@@ -430,8 +470,10 @@ dequantize_v5_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restri
             tma_store_3d(&tmo, 0, 0, (int)(j * 32), ob);
             tma_store_3d(&tmo, 0, 1, (int)(j * 32), ob + kChunkBytes5 / 2);
             bulk_commit();
+            // every code and norm read from the slot has been consumed (the
+            // staged output depends on them): refill it
+            if (j + (int64_t)kNSD5 * kW5 < c1) issue(j + (int64_t)kNSD5 * kW5, s);
         }
-        nrm = nrm_next;
     }
     if (lane == 0) bulk_wait<0>();
 }
@@ -451,7 +493,7 @@ __host__ __device__ inline int pair_copies5(int pw) { return pw <= 3 ? 16 : (pw 
 
 __host__ __device__ inline size_t dequantize_v5p_smem(int pw)
 {
-    return 1024 + (size_t)kW5 * kChunkBytes5 + (size_t)kW5 * kNSD5 * 512 * pw +
+    return 1024 + (size_t)kW5 * kChunkBytes5 + (size_t)kW5 * kNSD5 * (512 * pw + 64) +
            ((size_t)1 << (2 * pw)) * pair_copies5(pw) * 8 + 256 + 8 * kW5 * kNSD5;
 }
 
@@ -502,14 +544,15 @@ dequantize_v5p_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restr
 {
     static_assert(PW <= 5, "pair table of 2^(2 PW) entries");
     constexpr int CB = 16 * PW;
-    constexpr uint32_t RING = 512u * PW;
+    constexpr uint32_t RING = 512u * PW;              // one chunk's codes
+    constexpr uint32_t SLOT = RING + 64u;             // ... and its 32 fp16 norms
     constexpr int NE = 1 << (2 * PW);               // centroid pairs
     constexpr int CP = PW <= 4 ? 16 : 4;            // copies (lane % CP reads its own)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *outb = base;
     uint8_t *cring = outb + (size_t)kW5 * kChunkBytes5;
-    float2 *ptab = reinterpret_cast<float2 *>(cring + (size_t)kW5 * kNSD5 * RING);
+    float2 *ptab = reinterpret_cast<float2 *>(cring + (size_t)kW5 * kNSD5 * SLOT);
     uint32_t *pmask = reinterpret_cast<uint32_t *>(ptab + NE * CP);
     uint64_t *full = reinterpret_cast<uint64_t *>(pmask + 64);
 
@@ -529,13 +572,22 @@ dequantize_v5p_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restr
     setup_pair_masks(T, pmask, 128);
     __syncthreads();
 
-    uint8_t *wring = cring + (size_t)warp * kNSD5 * RING;
+    uint8_t *wring = cring + (size_t)warp * kNSD5 * SLOT;
     uint8_t *wout = outb + (size_t)warp * kChunkBytes5;
     uint64_t *wfull = full + warp * kNSD5;
+    // the chunk's codes and the whole 16-byte groups of its norms (the norms
+    // of a ragged last chunk's remaining blocks are read from global memory)
+    auto norm_bytes = [&](int64_t j) -> uint32_t {
+        const int64_t nb = nblocks - j * 32 < 32 ? nblocks - j * 32 : 32;
+        return (uint32_t)(nb * 2) & ~15u;
+    };
     auto issue = [&](int64_t j, int s) {
         const int64_t nb = nblocks - j * 32 < 32 ? nblocks - j * 32 : 32;
-        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(nb * CB));
-        bulk_load(wring + (size_t)s * RING, codes + j * 32 * CB, (uint32_t)(nb * CB), &wfull[s]);
+        const uint32_t nbytes = norm_bytes(j);
+        fence_proxy_async_smem();                   // the slot's earlier generic reads precede the copy
+        mbar_arrive_expect_tx(&wfull[s], (uint32_t)(nb * CB) + nbytes);
+        bulk_load(wring + (size_t)s * SLOT, codes + j * 32 * CB, (uint32_t)(nb * CB), &wfull[s]);
+        if (nbytes) bulk_load(wring + (size_t)s * SLOT + RING, norms + j * 32, nbytes, &wfull[s]);
     };
     if (lane == 0)
         for (int s = 0; s < kNSD5; ++s) {
@@ -544,27 +596,32 @@ dequantize_v5p_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restr
         }
     const uint32_t ptab_lane = smem_u32(ptab) + (uint32_t)(lane & (CP - 1)) * 8u;
     const uint32_t pm = smem_u32(pmask);
-    auto fetch_norm = [&](int64_t j) -> float {
-        const int64_t blk = j * 32 + lane;
-        return (j < c1 && blk < nblocks) ? h16_to_f32(__ldg(norms + blk)) : 0.0f;
-    };
-    float nrm = fetch_norm(c0 + warp);
 
     for (int64_t k = 0;; ++k) {
         const int64_t j = c0 + warp + k * kW5;
         if (j >= c1) break;
         const int s = (int)(k % kNSD5);
-        const float nrm_next = fetch_norm(j + kW5);
         if (!mbar_wait(&wfull[s], (uint32_t)((k / kNSD5) & 1))) break;
+        float nrm;
+        {
+            const int64_t blk = j * 32 + lane;
+            uint16_t h = 0;
+            if ((uint32_t)lane * 2u < norm_bytes(j)) {
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(h)
+                             : "r"(smem_u32(wring + (size_t)s * SLOT + RING) + (uint32_t)lane * 2u));
+            } else if (blk < nblocks) {
+                h = __ldg(norms + blk);
+            }
+            nrm = h16_to_f32(h);
+        }
         uint32_t cw[4 * PW];
-        const uint32_t src = smem_u32(wring + (size_t)s * RING) + (uint32_t)lane * CB;
+        const uint32_t src = smem_u32(wring + (size_t)s * SLOT) + (uint32_t)lane * CB;
 #pragma unroll
         for (int q = 0; q < PW; ++q) {
-            const uint4 v = lds128(src + 16u * q);
+            const uint4 v = lds128_fresh(src + 16u * q);
             cw[4 * q] = v.x; cw[4 * q + 1] = v.y; cw[4 * q + 2] = v.z; cw[4 * q + 3] = v.w;
         }
-        __syncwarp();
-        if (lane == 0 && j + (int64_t)kNSD5 * kW5 < c1) issue(j + (int64_t)kNSD5 * kW5, s);
         float2 Q[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
@@ -588,8 +645,10 @@ dequantize_v5p_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restr
             tma_store_3d(&tmo, 0, 0, (int)(j * 32), ob);
             tma_store_3d(&tmo, 0, 1, (int)(j * 32), ob + kChunkBytes5 / 2);
             bulk_commit();
+            // every code and norm read from the slot has been consumed (the
+            // staged output depends on them): refill it
+            if (j + (int64_t)kNSD5 * kW5 < c1) issue(j + (int64_t)kNSD5 * kW5, s);
         }
-        nrm = nrm_next;
     }
     if (lane == 0) bulk_wait<0>();
 }

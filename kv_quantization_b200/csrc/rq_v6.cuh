@@ -61,12 +61,12 @@ __device__ __forceinline__ void sign_fold_projection(uint8_t *s_S, int m16, cons
 }
 
 template <bool BF16, bool SIGNS>
-__device__ __forceinline__ void load_half64(uint32_t row_base, int blk, uint32_t pmask_half, float2 *P, bool fresh)
+__device__ __forceinline__ void load_half64(uint32_t row_base, int blk, uint32_t pmask_half, float2 *P)
 {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        uint4 a = fresh ? lds128_fresh(row_base + sw128_offset(blk, k)) : lds128(row_base + sw128_offset(blk, k));
-        uint4 b = fresh ? lds128_fresh(row_base + sw128_offset(blk, k + 4)) : lds128(row_base + sw128_offset(blk, k + 4));
+        uint4 a = lds128_fresh(row_base + sw128_offset(blk, k));
+        uint4 b = lds128_fresh(row_base + sw128_offset(blk, k + 4));
         if constexpr (SIGNS) {
             const uint4 ma = lds128_fresh(pmask_half + 16u * k);
             const uint4 mb = lds128_fresh(pmask_half + 16u * (k + 4));
@@ -345,7 +345,7 @@ qjl_v6_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
         const bool valid = blk < nblocks;
 
         float2 P[32];
-        load_half64<BF16, SIGNS>(rbase, blk_row, pmh, P, false);
+        load_half64<BF16, SIGNS>(rbase, blk_row, pmh, P);
         const float n32 = __fsqrt_rn(sumsq_half64(P));
         fwht_half64(P, hf);
         const float inv = n32 > 0.0f ? __frcp_rn(n32) : 0.0f;

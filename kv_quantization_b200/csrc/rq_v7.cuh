@@ -138,7 +138,7 @@ qjl_v7_quant_kernel(const __grid_constant__ CUtensorMap tmx, int64_t nblocks, co
         const bool valid = blk < nblocks;
 
         float2 P[32];
-        load_half64<BF16, SIGNS>(rbase, blk_row, pmq, P, false);
+        load_half64<BF16, SIGNS>(rbase, blk_row, pmq, P);
         const float n32 = __fsqrt_rn(sumsq_half64<4, 8>(P));
         fwht_half64<4, 8>(P, q);
         const float inv = n32 > 0.0f ? __frcp_rn(n32) : 0.0f;

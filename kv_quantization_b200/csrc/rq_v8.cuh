@@ -149,7 +149,7 @@ qjl_v8_quant_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_consta
             const int64_t blk = t * 128 + blk_row;
             const bool valid = blk < nblocks;
             float2 P[32];
-            load_half64<BF16, SIGNS>(rbase, blk_row, pmq, P, false);
+            load_half64<BF16, SIGNS>(rbase, blk_row, pmq, P);
             const float n32 = __fsqrt_rn(sumsq_half64<8, 4>(P));
             fwht_half64<8, 4>(P, q);
             const float inv = n32 > 0.0f ? __frcp_rn(n32) : 0.0f;

@@ -83,6 +83,34 @@ def test_weight_4096sq_fused_qjl_full_size(bits):
                        f"weight4096sq b{bits}")
 
 
+@pytest.mark.parametrize("bits", [3, 4, 5])
+def test_weight_4096sq_every_block_fresh_buffers(bits):
+    """Quantize then dequantize the 4096 x 4096 weight into freshly allocated,
+    sentinel-filled buffers, twice, and compare every block with the oracle:
+    a read of shared memory that ran ahead of the bulk copy filling it would
+    show up here as stale data in the first pass after new codes."""
+    d = 128
+    x = synth.student_t_outliers(4096, 4096, seed=1, device=DEV).reshape(-1)
+    n = x.numel()
+    cent = L.rq_lloyd_max(bits)
+    x16 = u16(x)
+    s = O.sign_diagonal(1, d)
+    oc, on, _, _ = O.quantize(x16, O.BF16, d, bits, O.PACKED, s, cent)
+    for trial in range(2):
+        codes = torch.full((L.rq_code_bytes(n, d, bits, L.RQ_CODES_PACKED),), 0x5A, dtype=torch.uint8, device=DEV)
+        norms = torch.full((n // d,), 0x3C00, dtype=torch.int16, device=DEV)
+        L.rq_quantize(x, d, bits, L.RQ_CODES_PACKED, 1, 1, cent, codes, norms)
+        out = torch.full_like(x, float("nan"))
+        L.rq_dequantize(codes, norms, n, d, bits, L.RQ_CODES_PACKED, 1, 1, cent, out)
+        torch.cuda.synchronize()
+        gc = codes.cpu().numpy()
+        nmis = check_codes(gc, oc, x16, O.BF16, d, bits, O.PACKED, s, cent)
+        assert np.array_equal(norms.cpu().numpy().view(np.uint16), on)
+        oo, _ = O.dequantize(gc, on, d, bits, O.PACKED, s, cent, O.BF16)
+        assert np.array_equal(u16(out), oo), f"trial {trial}: {int((u16(out) != oo).sum())} values differ"
+        report("weight4096sq_full", bits=bits, trial=trial, code_mismatch=int(nmis))
+
+
 def sampled_tokens(G, T, sms, rng):
     """(group, token) pairs: the sampled units of the flat [G*T] key array,
     regrouped as the same token set for every group (scores compare on a
