@@ -564,7 +564,7 @@ def cpu_info():
     return model, os.cpu_count()
 
 
-def oracle_llama_sample(frac=8):
+def oracle_llama_sample(frac=1):
     """The first 1/frac of each of layer 0's seven matrices (the same seeded
     values the device arm quantizes), as bf16 bit patterns."""
     from kv_quantization_b200 import synth
@@ -597,7 +597,7 @@ def cpu_baseline():
     oracle_pair(x16)
     dt = time.perf_counter() - t0
     res = {"value": round(x16.size * 2 / dt / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-           "sample": f"first 1/8 of each of layer 0's seven matrices ({x16.size} values), 4-bit quantize + "
+           "sample": f"all of layer 0's seven matrices ({x16.size} values), 4-bit quantize + "
                      f"dequantize, {dt:.1f} s on one thread",
            "cpu_model": model, "nproc": ncpu, "per_workload": {}}
     pw = res["per_workload"]
