@@ -69,6 +69,9 @@ def lib():
                 "orc_sketch": (i32, [u16, i32, i64, i32, i32, u16, u8, f64]),
                 "orc_score": (i32, [u16, i64, i32, i32, i32, u16, i32, u8, u16, i64,
                                     u8, u16, i32, i32, i8, f32, f64]),
+                "orc_attention": (i32, [u16, i64, i32, i32, i32, u16, i32, u8, u16, i64,
+                                        u8, u16, i32, i32, i8, f32,
+                                        u8, u16, i32, i32, i8, f32, C.c_double, f64]),
                 "orc_unpack_codes": (None, [u8, i64, i32, i32, i32, u8]),
                 "orc_pack_codes": (None, [u8, i64, i32, i32, i32, u8]),
                 "orc_hadamard_matrix": (None, [i32, f64]),
@@ -247,6 +250,35 @@ def score(q16, G, nq, d, m, S16, sdtype, signs, sk_norms, T, codes=None, norms=N
                     _ptr(cd, C.c_uint8), _ptr(nr, C.c_uint16), bits, layout,
                     _ptr(s, C.c_int8), _ptr(cc, C.c_float), _ptr(out, C.c_double))
     return out.reshape(G, nq, T)
+
+
+def attention(q16, G, nq, d, m, S16, sdtype, signs, sk_norms, T, vcodes, vnorms, vbits, vlayout, vsigns_diag,
+              vc32, softmax_scale, codes=None, norms=None, bits=0, layout=PACKED, signs_diag=None, c32=None):
+    """orc_attention -> fp64 [G][nq][d]: softmax(scale * score) over the T
+    keys of each group, applied to the fp64 reconstructions of the values."""
+    q16 = _u16(q16).reshape(-1)
+    S16 = _u16(S16).reshape(-1)
+    signs = np.ascontiguousarray(signs, np.uint8)
+    sk_norms = _u16(sk_norms)
+    cd = None if codes is None else np.ascontiguousarray(codes, np.uint8)
+    nr = None if norms is None else _u16(norms)
+    cc = None if c32 is None else np.ascontiguousarray(c32, np.float32)
+    s = _signs_arr(signs_diag)
+    vcd = np.ascontiguousarray(vcodes, np.uint8)
+    vnr = _u16(vnorms)
+    vcc = np.ascontiguousarray(vc32, np.float32)
+    vs = _signs_arr(vsigns_diag)
+    out = np.zeros(G * nq * d, np.float64)
+    rc = lib().orc_attention(_ptr(q16, C.c_uint16), G, nq, d, m, _ptr(S16, C.c_uint16), sdtype,
+                             _ptr(signs, C.c_uint8), _ptr(sk_norms, C.c_uint16), T,
+                             _ptr(cd, C.c_uint8), _ptr(nr, C.c_uint16), bits, layout,
+                             _ptr(s, C.c_int8), _ptr(cc, C.c_float),
+                             _ptr(vcd, C.c_uint8), _ptr(vnr, C.c_uint16), vbits, vlayout,
+                             _ptr(vs, C.c_int8), _ptr(vcc, C.c_float), float(softmax_scale),
+                             _ptr(out, C.c_double))
+    if rc != 0:
+        raise ValueError("orc_attention: empty key range")
+    return out.reshape(G, nq, d)
 
 
 def unpack_codes(codes, nblocks, d, bits, layout):

@@ -559,6 +559,54 @@ int orc_score(const uint16_t *q, int64_t G, int nq, int d, int m, const uint16_t
 }
 
 /* Explicit d x d Sylvester Hadamard matrix (entries +-1), for tests. */
+/* Attention decode over compressed keys and values.  The QJL page ("QJL",
+ * "What this is -- and what it is NOT" and "Algorithm in one paragraph")
+ * pairs 1-bit JL keys with TurboQuant 4-bit values and reconstructs each
+ * query-key score at attention time; the GLQ page ("KV cache compression",
+ * "Inline-dequant E8 KV") dequantizes K/V inside the attention kernel with
+ * the inverse Hadamard and splits the key range for long contexts.  The
+ * attention itself is the standard one:
+ *   out[g][q][:] = sum_t p_t * vh_t,  p_t = exp(a_t - max_u a_u) / sum_u exp(a_u - max_u a_u),
+ *   a_t = softmax_scale * score[g][q][t]
+ * with score the estimator of orc_score and vh_t the fp64 reconstruction of
+ * value block (g, t) (orc_dequantize_f64).  fp64 throughout.  Arguments as
+ * orc_score for the keys; vcodes/vnorms [G][T] blocks of d with their own
+ * bits, layout, sign diagonal and table; out fp64 [G][nq][d]. */
+int orc_attention(const uint16_t *q, int64_t G, int nq, int d, int m, const uint16_t *S, int sdtype,
+                  const uint8_t *signs, const uint16_t *sk_norms, int64_t T,
+                  const uint8_t *codes, const uint16_t *norms, int bits, int layout,
+                  const int8_t *s, const float *c,
+                  const uint8_t *vcodes, const uint16_t *vnorms, int vbits, int vlayout,
+                  const int8_t *vs, const float *vc, double softmax_scale, double *out)
+{
+    if (T <= 0) return -1;
+    double *sc = (double *)malloc(sizeof(double) * (size_t)nq * (size_t)T);
+    double *vh = (double *)malloc(sizeof(double) * (size_t)T * (size_t)d);
+    int64_t cb = codes ? block_code_bytes(d, bits, layout) : 0;
+    int64_t vcb = block_code_bytes(d, vbits, vlayout);
+    int mb = m / 8;
+    for (int64_t g = 0; g < G; ++g) {
+        orc_score(q + g * nq * d, 1, nq, d, m, S, sdtype, signs + g * T * mb, sk_norms + g * T, T,
+                  codes ? codes + g * T * cb : NULL, norms ? norms + g * T : NULL, bits, layout, s, c, sc);
+        orc_dequantize_f64(vcodes + g * T * vcb, vnorms + g * T, T, d, vbits, vlayout, vs, vc, vh);
+        for (int qi = 0; qi < nq; ++qi) {
+            const double *a = sc + (int64_t)qi * T;
+            double mx = -INFINITY;
+            for (int64_t t = 0; t < T; ++t) if (softmax_scale * a[t] > mx) mx = softmax_scale * a[t];
+            double l = 0.0;
+            for (int64_t t = 0; t < T; ++t) l += exp(softmax_scale * a[t] - mx);
+            double *o = out + (g * nq + qi) * d;
+            for (int j = 0; j < d; ++j) o[j] = 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                double p = exp(softmax_scale * a[t] - mx) / l;
+                for (int j = 0; j < d; ++j) o[j] += p * vh[t * d + j];
+            }
+        }
+    }
+    free(sc); free(vh);
+    return 0;
+}
+
 void orc_hadamard_matrix(int d, double *H)
 {
     for (int i = 0; i < d; ++i)

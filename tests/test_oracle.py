@@ -387,3 +387,110 @@ def test_score_first_stage_equals_dot_with_reconstruction():
     xh = O.dequantize_f64(codes, norms, d, bits, O.PACKED, s, c).reshape(n, d)
     qf = (q.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(nq, d)
     assert np.allclose(sc, qf @ xh.T, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ attention over compressed K/V
+
+def _attn_case(rng, G, T, nq, d, m, kbits, vbits, two_stage=True):
+    """Keys (two-stage or pure QJL) and 4-bit values of G groups, compressed
+    by the oracle; returns the arguments of O.attention and the pieces a pin
+    needs."""
+    kc, vc = O.f32_table(kbits), O.f32_table(vbits)
+    ks, vs = O.sign_diagonal(21, d), O.sign_diagonal(22, d)
+    S = O.projection(23, m, d, O.BF16)
+    k = rand_u16(rng, G * T * d, 1.0, O.BF16)
+    v = rand_u16(rng, G * T * d, 1.0, O.BF16)
+    q = rand_u16(rng, G * nq * d, 1.0, O.BF16)
+    if two_stage:
+        codes, norms, _, _ = O.quantize(k, O.BF16, d, kbits, O.PACKED, ks, kc)
+        r, rn = O.residual(k, O.BF16, codes, norms, d, kbits, O.PACKED, ks, kc)
+        sg, _ = O.sketch(r, O.BF16, d, m, S)
+        kw = dict(codes=codes, norms=norms, bits=kbits, layout=O.PACKED, signs_diag=ks, c32=kc)
+    else:
+        sg, _ = O.sketch(k, O.BF16, d, m, S)
+        rn = O.vec_norms(k, O.BF16, d)
+        kw = {}
+    vcodes, vnorms, _, _ = O.quantize(v, O.BF16, d, vbits, O.PACKED, vs, vc)
+    return dict(q=q, S=S, sg=sg, rn=rn, kw=kw, vcodes=vcodes, vnorms=vnorms, vs=vs, vc=vc)
+
+
+def _attn(c, G, nq, d, m, T, vbits, scale, **over):
+    a = dict(c)
+    a.update(over)
+    return O.attention(a["q"], G, nq, d, m, a["S"], O.BF16, a["sg"], a["rn"], T, a["vcodes"], a["vnorms"], vbits,
+                       O.PACKED, a["vs"], a["vc"], scale, **a["kw"])
+
+
+@pytest.mark.parametrize("two_stage", [True, False])
+def test_attention_matches_scipy_softmax_of_scores(two_stage):
+    """softmax(scale * score) @ V with scipy's softmax and numpy's product over
+    the oracle's own (pinned) scores and fp64 reconstructions: fixes the
+    scale, the per-group key/value offsets and the normalisation."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(30)
+    G, T, nq, d, m, vbits = 3, 37, 5, 64, 64, 4
+    c = _attn_case(rng, G, T, nq, d, m, 2, vbits, two_stage)
+    scale = 1.0 / math.sqrt(d)
+    got = _attn(c, G, nq, d, m, T, vbits, scale)
+    sc = O.score(c["q"], G, nq, d, m, c["S"], O.BF16, c["sg"], c["rn"], T, **c["kw"])
+    vh = O.dequantize_f64(c["vcodes"], c["vnorms"], d, vbits, O.PACKED, c["vs"], c["vc"]).reshape(G, T, d)
+    want = np.einsum("gqt,gtd->gqd", softmax(scale * sc, axis=-1), vh)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_single_key_returns_its_value():
+    rng = np.random.default_rng(31)
+    G, T, nq, d, m, vbits = 2, 1, 3, 128, 128, 4
+    c = _attn_case(rng, G, T, nq, d, m, 3, vbits)
+    got = _attn(c, G, nq, d, m, T, vbits, 0.125)
+    vh = O.dequantize_f64(c["vcodes"], c["vnorms"], d, vbits, O.PACKED, c["vs"], c["vc"]).reshape(G, 1, d)
+    assert np.array_equal(got, np.broadcast_to(vh, (G, nq, d)))
+
+
+def test_attention_equal_keys_average_the_values():
+    """Every key of a group identical: the weights are uniform whatever the
+    scores, so the output is the plain mean of the reconstructed values."""
+    rng = np.random.default_rng(32)
+    G, T, nq, d, m, vbits = 2, 20, 4, 64, 64, 3
+    c = _attn_case(rng, G, T, nq, d, m, 2, vbits)
+    mb = m // 8
+    for key in ("sg", "rn"):
+        arr = c[key].reshape(G, T, -1)
+        c[key] = np.ascontiguousarray(np.repeat(arr[:, :1], T, axis=1)).reshape(-1)
+    cb = O.code_bytes_per_block(d, 2, O.PACKED)
+    c["kw"]["codes"] = np.ascontiguousarray(np.repeat(c["kw"]["codes"].reshape(G, T, cb)[:, :1], T, axis=1)).reshape(-1)
+    c["kw"]["norms"] = np.ascontiguousarray(np.repeat(c["kw"]["norms"].reshape(G, T)[:, :1], T, axis=1)).reshape(-1)
+    assert c["sg"].size == G * T * mb
+    got = _attn(c, G, nq, d, m, T, vbits, 0.3)
+    vh = O.dequantize_f64(c["vcodes"], c["vnorms"], d, vbits, O.PACKED, c["vs"], c["vc"]).reshape(G, T, d)
+    want = np.broadcast_to(vh.mean(axis=1)[:, None, :], (G, nq, d))
+    assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+def test_attention_token_permutation_invariant_and_hard_limit():
+    """Permuting the tokens (keys and values together) leaves the output
+    unchanged; a very large scale selects the value of the top-scoring key
+    (and the max subtraction keeps it finite)."""
+    rng = np.random.default_rng(33)
+    G, T, nq, d, m, vbits, kbits = 1, 29, 4, 64, 64, 4, 2
+    c = _attn_case(rng, G, T, nq, d, m, kbits, vbits)
+    base = _attn(c, G, nq, d, m, T, vbits, 0.2)
+    perm = rng.permutation(T)
+    mb, cb, vcb = m // 8, O.code_bytes_per_block(d, kbits, O.PACKED), O.code_bytes_per_block(d, vbits, O.PACKED)
+    p = dict(c)
+    p["sg"] = np.ascontiguousarray(c["sg"].reshape(T, mb)[perm]).reshape(-1)
+    p["rn"] = np.ascontiguousarray(c["rn"][perm])
+    p["vcodes"] = np.ascontiguousarray(c["vcodes"].reshape(T, vcb)[perm]).reshape(-1)
+    p["vnorms"] = np.ascontiguousarray(c["vnorms"][perm])
+    p["kw"] = dict(c["kw"])
+    p["kw"]["codes"] = np.ascontiguousarray(c["kw"]["codes"].reshape(T, cb)[perm]).reshape(-1)
+    p["kw"]["norms"] = np.ascontiguousarray(c["kw"]["norms"][perm])
+    assert np.allclose(_attn(p, G, nq, d, m, T, vbits, 0.2), base, rtol=1e-12, atol=1e-12)
+    sc = O.score(c["q"], G, nq, d, m, c["S"], O.BF16, c["sg"], c["rn"], T, **c["kw"])[0]
+    top = np.argsort(sc, axis=1)
+    gap = sc[np.arange(nq), top[:, -1]] - sc[np.arange(nq), top[:, -2]]
+    scale = 800.0 / gap.min()
+    hard = _attn(c, G, nq, d, m, T, vbits, scale)[0]
+    vh = O.dequantize_f64(c["vcodes"], c["vnorms"], d, vbits, O.PACKED, c["vs"], c["vc"]).reshape(T, d)
+    assert np.all(np.isfinite(hard))
+    assert np.allclose(hard, vh[top[:, -1]], rtol=0, atol=1e-12)
