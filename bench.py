@@ -59,7 +59,7 @@ def parse(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile", default=None,
                    help="run one case's kernels once (profiling driver): c3_layer, weight4096_fused, kv_sketch, "
-                        "kv_score, kv_v, tq256, tq512; print nothing else")
+                        "kv_score, kv_attention, kv_v, tq256, tq512; print nothing else")
     p.add_argument("--rank-selftest", action="store_true", help=argparse.SUPPRESS)
     return p.parse_args(argv)
 
@@ -420,7 +420,8 @@ def secondary_lines(dev, reps=10, only=None):
     from kv_quantization_b200 import synth
     flush = l2_flusher(dev)
     out = []
-    want = (lambda k: True) if only is None else (lambda k: k == only)
+    # the attention line runs on the key line's sketch, so it comes with it
+    want = (lambda k: True) if only is None else (lambda k: k == only or (only == "kv_k" and k == "kv_attn"))
 
     if want("c1"):
         # 256 x 512 fp16, d = 128, 4-bit int8 codes, no signs: L2-resident latency
@@ -507,7 +508,33 @@ def secondary_lines(dev, reps=10, only=None):
                     "sketch_roofline": roofline_hbm(kbytes, tk, flops=2 * m * d * G * T),
                     "score_roofline": roofline_hbm(sbytes, ts, note="signs + norms read, fp32 scores written; "
                                                                     "query prologue included")})
-        del k, signs, kn, scores, ws
+        del scores, ws
+        if want("kv_attn"):
+            # attention decode over the sketched keys and the 4-bit values of the V line's recipe
+            v = synth.kv_with_channels(4, 8, T, d, seed=13, device=dev).reshape(-1)
+            vc = rq.rq_lloyd_max(4)
+            vcodes = torch.empty(G * T * d // 2, dtype=torch.uint8, device=dev)
+            vnorms = torch.empty(G * T, dtype=torch.int16, device=dev)
+            rq.rq_quantize(v, d, 4, rq.RQ_CODES_PACKED, 1, 14, vc, vcodes, vnorms)
+            del v
+            aout = torch.empty(G, nq, d, dtype=torch.float32, device=dev)
+            aws = torch.empty((rq.qjl_attention_workspace_bytes(G, nq, d, m, T) + 3) // 4, dtype=torch.float32,
+                              device=dev)
+            at = lambda: rq.qjl_attention(q, G, nq, d, m, S, signs, kn, T, vcodes, vnorms, 4, vc, aout, aws,
+                                          1.0 / d ** 0.5, v_use_signs=1, v_sign_seed=14)
+            at()
+            ta = median_ms(at, reps, flush)
+            abytes = signs.numel() + kn.numel() * 2 + vcodes.numel() + vnorms.numel() * 2 + q.numel() * 2 + \
+                aout.numel() * 4
+            out.append({"workload": "KV cache 4x8x32768x128 attention decode: the pure-QJL keys above (m=256) and "
+                                    "4-bit values (signs seed 14), 32 queries per (batch, head), softmax scale "
+                                    "1/sqrt(128); prologue + fused score/softmax/PV kernel + combine",
+                        "attention_ms": round(ta, 4), "token_heads_per_s": round(G * T / (ta * 1e-3), 1),
+                        "unfused_score_ms_for_context": round(ts, 4),
+                        "roofline": roofline_hbm(abytes, ta, note="key signs + norms, value codes + norms read once; "
+                                                                  "queries and outputs")})
+            del vcodes, vnorms, aout, aws
+        del k, signs, kn
 
     for d, seed in ((256, 6), (512, 8)):
         if not want(f"tq{d}"):
@@ -635,6 +662,14 @@ def cpu_baseline():
     t0 = time.perf_counter()
     O.score(q16, 1, 32, 128, 256, S, O.BF16, sg[: 4096 * 32], kn[:4096], 4096)
     pw["kv_score_token_heads_per_s"] = round(4096 / (time.perf_counter() - t0), 1)
+    # attention decode: 32 queries over 2048 sketched keys and 4-bit values of one head
+    v16 = synth.as_u16(synth.kv_with_channels(1, 1, 2048, 128, seed=13, device="cpu")).reshape(-1)
+    vs = O.sign_diagonal(14, 128)
+    vcd, vnr, _, _ = O.quantize(v16, O.BF16, 128, 4, O.PACKED, vs, c4)
+    t0 = time.perf_counter()
+    O.attention(q16, 1, 32, 128, 256, S, O.BF16, sg[: 2048 * 32], kn[:2048], 2048, vcd, vnr, 4, O.PACKED, vs, c4,
+                1.0 / 128 ** 0.5)
+    pw["kv_attention_token_heads_per_s"] = round(2048 / (time.perf_counter() - t0), 1)
     # TurboQuant-style keys at d = 256 / 512: compress 2048 keys, score 32 queries over 2048 keys
     for d in (256, 512):
         kk = synth.normal((1, 2048, d), seed=6, device="cpu").reshape(-1)
@@ -702,8 +737,8 @@ def profile_case(case):
         rq.rq_quantize(x, D, BITS, rq.RQ_CODES_PACKED, 1, 1000, cent, codes, norms)
         rq.rq_dequantize(codes, norms, LAYER_N, D, BITS, rq.RQ_CODES_PACKED, 1, 1000, cent, out)
     else:
-        key = {"weight4096_fused": "weight4096", "kv_sketch": "kv_k", "kv_score": "kv_k", "kv_v": "kv_v",
-               "tq256": "tq256", "tq512": "tq512"}[case]
+        key = {"weight4096_fused": "weight4096", "kv_sketch": "kv_k", "kv_score": "kv_k", "kv_attention": "kv_k",
+               "kv_v": "kv_v", "tq256": "tq256", "tq512": "tq512"}[case]
         secondary_lines(dev, reps=1, only=key)
     torch.cuda.synchronize()
     assert rq.rq_device_error(True) == 0

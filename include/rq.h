@@ -181,6 +181,44 @@ rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void 
                     int use_signs, uint64_t sign_seed, const float *centroids,
                     float *scores, void *workspace, size_t workspace_bytes, rq_stream_t stream);
 
+/* Device workspace qjl_attention needs (bytes), for the current device. */
+size_t qjl_attention_workspace_bytes(int64_t G, int n_q, int d, int m, int64_t T);
+
+/* Attention decode over compressed keys and values.  The QJL page ("QJL",
+ * "What this is -- and what it is NOT") pairs 1-bit JL keys with 4-bit
+ * TurboQuant values and ("Algorithm in one paragraph") rebuilds each
+ * query-key score at attention time from the same projection; the GLQ page
+ * ("KV cache compression", "Inline-dequant E8 KV") dequantizes K/V inside the
+ * attention kernel, with the inverse Hadamard and a split of the key range for
+ * long contexts.  For every group g and query i:
+ *   out[g][i][:] = sum_t p_t vh_t,  p_t = softmax over t of softmax_scale * s(i, t),
+ * s the qjl_score estimator of the keys (pure QJL when codes == NULL, else
+ * two-stage) and vh_t the reconstruction of value block (g, t) that
+ * rq_dequantize computes before its 16-bit rounding:
+ *   vh_t = D_v H (c_v[v_codes_t] * v_norms_t / d).
+ *   q, proj, signs, sk_norms, codes, norms, bits, layout, use_signs,
+ *   sign_seed, centroids: as qjl_score;
+ *   v_codes [G][T] blocks of d (v_layout), v_norms fp16 [G][T], with their
+ *   own v_bits, v_use_signs, v_sign_seed and v_centroids (rq_quantize's
+ *   arguments for the values);
+ *   out: fp32 [G][n_q][d] (caller-owned);
+ *   workspace: qjl_attention_workspace_bytes(G, n_q, d, m, T) bytes of device
+ *   memory (overwritten).
+ * Computed in fp32 with fp16 tensor-core operands: the scores as qjl_score,
+ * 2^x by the hardware approximation, the weights 2^14 p and the values
+ * c * (n / d) rounded to fp16 for the weighted sum.
+ * Supported: d = 128, n_q <= 32, m % 128 == 0, two-stage keys of 1, 2, 3, 4
+ * bits packed or int8 codes with d * width / 8 % 16 == 0, values of 2, 3, 4
+ * bits packed or int8; other valid shapes return RQ_EUNSUPPORTED.  T >= 1. */
+rq_status qjl_attention(const void *q, int64_t G, int n_q, int d, int m, const void *proj, rq_dtype proj_dtype,
+                        const uint8_t *signs, const uint16_t *sk_norms, int64_t T,
+                        const void *codes, const uint16_t *norms, int bits, rq_layout layout,
+                        int use_signs, uint64_t sign_seed, const float *centroids,
+                        const void *v_codes, const uint16_t *v_norms, int v_bits, rq_layout v_layout,
+                        int v_use_signs, uint64_t v_sign_seed, const float *v_centroids,
+                        float softmax_scale, float *out, void *workspace, size_t workspace_bytes,
+                        rq_stream_t stream);
+
 /* qjl_score without a caller-provided workspace.  The pages have no
  * counterpart to this entry point; it exists for callers that cannot allocate
  * device memory -- a serving engine that reserved all of its HBM for the KV

@@ -54,6 +54,9 @@ def lib() -> C.CDLL:
                 "qjl_score_workspace_bytes": (sz, [i64, i32, i32, i32]),
                 "qjl_score": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32, u64,
                                     fp, vp, vp, sz, vp]),
+                "qjl_attention_workspace_bytes": (sz, [i64, i32, i32, i32, i64]),
+                "qjl_attention": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32, u64,
+                                        vp, vp, vp, i32, i32, i32, u64, vp, C.c_float, vp, vp, sz, vp]),
                 "qjl_score_noalloc": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32,
                                             u64, fp, vp, vp]),
             }
@@ -69,7 +72,7 @@ def exported_symbols():
     """Names this binding expects librq.so to export."""
     return ["rq_status_string", "rq_device_error", "rq_last_launch", "rq_probe_bounded_wait", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
             "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score",
-            "qjl_score_noalloc"]
+            "qjl_score_noalloc", "qjl_attention_workspace_bytes", "qjl_attention"]
 
 
 def status_string(status: int) -> str:
@@ -176,6 +179,27 @@ def qjl_score(q, G, n_q, d, m, proj, signs, sk_norms, T, scores, workspace, code
     _check("qjl_score", lib().qjl_score(
         _dev(q), G, n_q, d, m, _dev(proj), _dtype_code(proj), _dev(signs), _dev(sk_norms), T, _dev(codes),
         _dev(norms), bits, layout, int(use_signs), sign_seed, cp, _dev(scores), _dev(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def qjl_attention_workspace_bytes(G, n_q, d, m, T) -> int:
+    return lib().qjl_attention_workspace_bytes(G, n_q, d, m, T)
+
+
+def qjl_attention(q, G, n_q, d, m, proj, signs, sk_norms, T, v_codes, v_norms, v_bits, v_centroids, out, workspace,
+                  softmax_scale, codes=None, norms=None, bits=0, layout=RQ_CODES_PACKED, use_signs=0, sign_seed=0,
+                  centroids=None, v_layout=RQ_CODES_PACKED, v_use_signs=0, v_sign_seed=0, stream=None):
+    """Softmax(softmax_scale * score) over the T compressed keys of each group,
+    applied to the in-kernel reconstructions of the compressed values:
+    out fp32 [G][n_q][d]."""
+    cp = None
+    if centroids is not None:
+        c, cp = _table(centroids)
+    vc, vcp = _table(v_centroids)
+    _check("qjl_attention", lib().qjl_attention(
+        _dev(q), G, n_q, d, m, _dev(proj), _dtype_code(proj), _dev(signs), _dev(sk_norms), T, _dev(codes),
+        _dev(norms), bits, layout, int(use_signs), sign_seed, cp, _dev(v_codes), _dev(v_norms), v_bits, v_layout,
+        int(v_use_signs), v_sign_seed, vcp, float(softmax_scale), _dev(out), _dev(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

@@ -11,7 +11,7 @@
 
 #include "rq_common.cuh"
 #include "rq_kernels.h"
-#include "qjl_score_v4.cuh"
+#include "qjl_score_v5.cuh"
 
 namespace rq {
 
@@ -162,6 +162,18 @@ score_kernel(const float *__restrict__ ws, int nq, int d, int m, const uint8_t *
             scores[((int64_t)g * nq + q0 + qi) * T_len + t] = __fadd_rn(__fmul_rn(a1, acc1[qi]), __fmul_rn(a2, acc2[qi]));
 }
 
+cudaError_t launch_score_prologue(const ScoreArgs &a, bool two, uint16_t *wsB, float *wsN, cudaStream_t st)
+{
+    const size_t psmem = sc2_prologue_smem(a.d);
+    cudaError_t e = cudaFuncSetAttribute(score_v2_prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    if (e != cudaSuccess) return e;
+    const unsigned zsl = (unsigned)((sc2_m64(a.m) + kSc2PrologueOut - 1) / kSc2PrologueOut);
+    score_v2_prologue<<<dim3((unsigned)a.G, (unsigned)((a.nq + kSc2PrologueQ - 1) / kSc2PrologueQ), zsl), 256, psmem, st>>>(
+        a.q, a.nq, a.d, a.m, static_cast<const uint16_t *>(a.proj), a.proj_bf16, *a.tables, two, wsB, wsN);
+    note_launch("score_v2_prologue");
+    return cudaGetLastError();
+}
+
 size_t score_workspace_bytes(int64_t G, int nq, int d, int m)
 {
     const size_t v1 = (size_t)G * (size_t)nq * (size_t)(d + m) * sizeof(float);
@@ -188,6 +200,26 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
     note_launch("score_v2_prologue");
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    // queries on M, 256 tokens on N (qjl_score_v5.cuh) when the records allow
+    // aligned bulk copies: the deepest rings that fit
+    if (sc5_eligible(a.nq, a.d, a.m, TWO, PW)) {
+        struct Cfg5 { int ring, nrec; };
+        const Cfg5 cfgs5[] = {{4, 3}, {4, 2}, {3, 2}, {2, 2}, {2, 1}};
+        const int64_t items5 = a.G * ((a.T + kSc5Tok - 1) / kSc5Tok);
+        const int64_t grid5 = items5 < (int64_t)a.num_sms ? items5 : (int64_t)a.num_sms;
+        for (const Cfg5 &c : cfgs5) {
+            const size_t smem5 = sc5_smem(a.nq, a.d, a.m, TWO, PW, c.ring, c.nrec);
+            if (smem5 > kMaxSmemPerBlock) continue;
+            auto kern5 = score_v5_kernel<PW, TWO>;
+            e = cudaFuncSetAttribute(kern5, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem5);
+            if (e != cudaSuccess) return e;
+            kern5<<<(unsigned)(grid5 > 0 ? grid5 : 1), kSc5Threads, smem5, st>>>(
+                wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms, a.T, a.G, a.codes, a.norms, *a.tables, a.scores,
+                c.ring, c.nrec);
+            note_launch("score_v5_kernel");
+            return cudaGetLastError();
+        }
+    }
     const int64_t items = a.G * ((a.T + 127) / 128);
     const int64_t grid = items < (int64_t)a.num_sms ? items : (int64_t)a.num_sms;
     // eight producer warps (qjl_score_v4.cuh): the deepest configuration that fits

@@ -50,6 +50,9 @@ __host__ __device__ inline size_t sc2_prologue_smem(int d)
     return ((size_t)kSc2PrologueQ * (d + 4) + (size_t)kSc2PrologueQ * d + kSc2PrologueQ) * sizeof(float);
 }
 
+// The prologue kernel is defined in one translation unit only (qjl.cu);
+// other users launch it through launch_score_prologue().
+#ifndef RQ_SCORE_PROLOGUE_EXTERN
 __global__ void __launch_bounds__(256)
 score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const uint16_t *__restrict__ proj,
                   bool proj_bf16, const __grid_constant__ QuantTables T, bool two, uint16_t *__restrict__ wsB,
@@ -148,5 +151,6 @@ score_v2_prologue(const uint16_t *__restrict__ q, int nq, int d, int m, const ui
                 __half_as_ushort(__float2half_rn(acc.y * pinv[qp + 1]));
     }
 }
+#endif  // RQ_SCORE_PROLOGUE_EXTERN
 
 }  // namespace rq

@@ -529,6 +529,67 @@ rq_status qjl_sketch(const void *x, rq_dtype dtype, int64_t n_vec, int d, int m,
     return cuda_status(rq::launch_sketch(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t qjl_attention_workspace_bytes(int64_t G, int n_q, int d, int m, int64_t T)
+{
+    if (G < 0 || n_q < 0 || d < 0 || m < 0 || T < 0) return 0;
+    const int sms = num_sms();
+    return rq::attention_workspace_bytes(G, n_q, d, m, T, sms > 0 ? sms : 1);
+}
+
+rq_status qjl_attention(const void *q, int64_t G, int n_q, int d, int m, const void *proj, rq_dtype proj_dtype,
+                        const uint8_t *signs, const uint16_t *sk_norms, int64_t T_len,
+                        const void *codes, const uint16_t *norms, int bits, rq_layout layout,
+                        int use_signs, uint64_t sign_seed, const float *centroids,
+                        const void *v_codes, const uint16_t *v_norms, int v_bits, rq_layout v_layout,
+                        int v_use_signs, uint64_t v_sign_seed, const float *v_centroids,
+                        float softmax_scale, float *out, void *workspace, size_t workspace_bytes,
+                        rq_stream_t stream)
+{
+    rq::begin_call();
+    if (!pow2_d(d)) return RQ_EINVAL;
+    if (m < 8 || m > 512 || m % 8) return RQ_EINVAL;
+    if (proj_dtype != RQ_F16 && proj_dtype != RQ_BF16) return RQ_EINVAL;
+    if (G < 0 || n_q < 0 || T_len < 0) return RQ_EINVAL;
+    if (!(softmax_scale == softmax_scale) || softmax_scale < 0.0f || softmax_scale > 1e30f) return RQ_EINVAL;
+    if (G > 65535 || n_q > 65535 || T_len > ((int64_t)1 << 31)) return RQ_ESIZE;
+    if (G == 0 || n_q == 0) return RQ_OK;
+    if (T_len == 0) return RQ_EINVAL;                       // softmax over no keys
+    rq_status s = check_common(0, d, v_bits, v_layout);
+    if (s) return s;
+    if (!q || !proj || !signs || !sk_norms || !v_codes || !v_norms || !out || !workspace) return RQ_EINVAL;
+    if (!aligned16(q) || !aligned16(proj) || !aligned16(signs) || !aligned16(sk_norms) || !aligned16(v_codes) ||
+        !aligned16(v_norms) || !aligned16(out) || !aligned16(workspace))
+        return RQ_EALIGN;
+    QuantTables T;
+    std::memset(&T, 0, sizeof(T));
+    int pw = 0;
+    if (codes) {
+        s = check_common(0, d, bits, layout);
+        if (s) return s;
+        if (!norms) return RQ_EINVAL;
+        if (!aligned16(codes) || !aligned16(norms)) return RQ_EALIGN;
+        s = tables_for(centroids, bits, d, use_signs, sign_seed, T);
+        if (s) return s;
+        pw = layout == RQ_CODES_INT8 ? 8 : bits;
+    }
+    QuantTables TV;
+    s = tables_for(v_centroids, v_bits, d, v_use_signs, v_sign_seed, TV);
+    if (s) return s;
+    const int vpw = v_layout == RQ_CODES_INT8 ? 8 : v_bits;
+    if (!rq::attention_supported(n_q, d, m, codes != nullptr, pw, vpw)) return RQ_EUNSUPPORTED;
+    rq::AttnArgs a{};
+    a.k.q = static_cast<const uint16_t *>(q); a.k.G = G; a.k.nq = n_q; a.k.d = d; a.k.m = m; a.k.proj = proj;
+    a.k.proj_bf16 = proj_dtype == RQ_BF16; a.k.signs = signs; a.k.sk_norms = sk_norms; a.k.T = T_len;
+    a.k.codes = static_cast<const uint8_t *>(codes); a.k.norms = norms; a.k.pw = pw; a.k.tables = &T;
+    a.vcodes = static_cast<const uint8_t *>(v_codes); a.vnorms = v_norms; a.vpw = vpw; a.vtables = &TV;
+    a.softmax_scale = softmax_scale; a.out = out; a.workspace = workspace;
+    a.num_sms = num_sms();
+    if (a.num_sms <= 0) return RQ_ECUDA;
+    a.k.num_sms = a.num_sms;
+    if (workspace_bytes < rq::attention_workspace_bytes(G, n_q, d, m, T_len, a.num_sms)) return RQ_ESIZE;
+    return cuda_status(rq::launch_attention(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char *rq_last_launch(void) { return rq::g_trace; }
 
 rq_status rq_probe_bounded_wait(uint32_t polls, rq_stream_t stream)

@@ -89,6 +89,25 @@ cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t st);
 cudaError_t launch_projection(uint64_t seed, int m, int d, bool bf16, void *proj, cudaStream_t st);
 cudaError_t launch_sketch(const SketchArgs &a, cudaStream_t st);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t st);
+// The tensor-core score prologue alone (workspace rows [q~/||q|| ; Sq/||q||]
+// in fp16 and ||q|| in fp32, qjl_score_v2.cuh) for another kernel to consume.
+cudaError_t launch_score_prologue(const ScoreArgs &a, bool two, uint16_t *wsB, float *wsN, cudaStream_t st);
+
+// Attention decode over compressed keys and values (qjl_attention.cuh).
+struct AttnArgs {
+    ScoreArgs k;               // queries, projection, keys (scores / workspace unused)
+    const uint8_t *vcodes;     // value codes [G][T] blocks of d
+    const uint16_t *vnorms;    // fp16 [G][T]
+    int vpw;                   // value code field width (bits, or 8 for int8)
+    const QuantTables *vtables;
+    float softmax_scale;
+    float *out;                // fp32 [G][nq][d]
+    void *workspace;
+    int num_sms;
+};
+bool attention_supported(int nq, int d, int m, bool two, int pw, int vpw);
+size_t attention_workspace_bytes(int64_t G, int nq, int d, int m, int64_t T, int num_sms);
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st);
 size_t score_workspace_bytes(int64_t G, int nq, int d, int m);
 size_t quantize_smem_bytes(int d, bool qjl);
 // Encode the [rows][64] 16-bit row view of `ptr` as a TMA map (256-row boxes,

@@ -141,7 +141,7 @@ def test_kv_cache_key_sketch_and_score_full_size():
     scores = torch.empty(G, nq, T, dtype=torch.float32, device=DEV)
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, signs, kn, T, scores, ws)
-    assert L.rq_last_launch() == "score_v2_prologue,score_v4_kernel"
+    assert L.rq_last_launch() == "score_v2_prologue,score_v5_kernel"
     torch.cuda.synchronize()
     rng = np.random.default_rng(7)
     sms = num_sms()
@@ -195,7 +195,7 @@ def test_turboquant_keys_full_size(d):
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits,
                 layout=L.RQ_CODES_PACKED, use_signs=1, sign_seed=4, centroids=cent)
-    assert L.rq_last_launch() == "score_v2_prologue,score_v4_kernel"
+    assert L.rq_last_launch() == "score_v2_prologue,score_v5_kernel"
     torch.cuda.synchronize()
     rng = np.random.default_rng(d)
     sms = num_sms()
@@ -283,12 +283,13 @@ def test_sketch_many_tiles(d, m, kernel):
     assert np.array_equal(take_rows(kn, keys, 1).reshape(-1).view(np.uint16), O.vec_norms(k16, O.BF16, d))
 
 
-@pytest.mark.parametrize("d,bits,m,nq", [(128, 4, 128, 32), (256, 2, 256, 20), (128, 3, 64, 144)])
-def test_score_many_tiles(d, bits, m, nq):
+@pytest.mark.parametrize("d,bits,m,nq,kernel", [(128, 4, 128, 32, "score_v5_kernel"), (256, 2, 256, 20, "score_v5_kernel"),
+                                                (128, 3, 64, 24, "score_v4_kernel"), (128, 3, 64, 144, "score_kernel")])
+def test_score_many_tiles(d, bits, m, nq, kernel):
     """Scores over 3 x SMs token tiles per group set (the score's chunk ring
     wraps many times), every tile sampled."""
     G = 3
-    T = num_sms() * 128 + 77
+    T = num_sms() * (256 if kernel == "score_v5_kernel" else 128) + 77
     k = synth.normal((G, T, d), seed=60 + d, device=DEV).reshape(-1)
     cent = L.rq_lloyd_max(bits)
     S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
@@ -299,6 +300,7 @@ def test_score_many_tiles(d, bits, m, nq):
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits,
                 layout=L.RQ_CODES_PACKED, use_signs=1, sign_seed=62, centroids=cent)
+    assert L.rq_last_launch().split(",")[-1] == kernel
     torch.cuda.synchronize()
     rng = np.random.default_rng(d + nq)
     toks = np.unique(np.concatenate([[0, T - 1], [rng.integers(t, min(T, t + 128)) for t in range(0, T, 128)]]))

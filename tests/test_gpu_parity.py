@@ -342,8 +342,17 @@ def make_two_stage(G, T, d, bits, m, layout, seed, sseed, pseed):
     return k, cent, S, codes, norms, qs, qn
 
 
-def score_kernels(nq):
-    return "score_v2_prologue,score_v4_kernel" if nq <= 128 else "score_prologue_kernel,score_kernel"
+def score_kernels(nq, d=128, m=256, bits=0, layout=L.RQ_CODES_PACKED):
+    """Kernels qjl_score launches: queries on M (score_v5) when n_q <= 128 and
+    every token's sign bytes (and code bytes, for two-stage keys) are a
+    multiple of 16; the 128-token tensor-core kernel (score_v4) for the other
+    n_q <= 128 shapes; the CUDA-core score above 128 queries."""
+    if nq > 128:
+        return "score_prologue_kernel,score_kernel"
+    pw = 8 if layout == L.RQ_CODES_INT8 else bits
+    if (m // 8) % 16 == 0 and (bits == 0 or (d * pw // 8) % 16 == 0):
+        return "score_v2_prologue,score_v5_kernel"
+    return "score_v2_prologue,score_v4_kernel"
 
 
 @pytest.mark.parametrize("nq", [32, 160])
@@ -400,7 +409,7 @@ def test_score_two_stage(d):
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits,
                 layout=L.RQ_CODES_PACKED, use_signs=1, sign_seed=4, centroids=cent)
-    assert L.rq_last_launch() == score_kernels(nq)
+    assert L.rq_last_launch() == score_kernels(nq, d, m, bits)
     torch.cuda.synchronize()
     q16 = u16(q)
     n16 = norms.cpu().numpy().view(np.uint16)
@@ -412,6 +421,8 @@ def test_score_two_stage(d):
 
 @pytest.mark.parametrize("d,bits,m,nq,layout", [(128, 4, 128, 40, L.RQ_CODES_INT8), (64, 3, 72, 7, L.RQ_CODES_PACKED),
                                                  (128, 5, 256, 33, L.RQ_CODES_PACKED),
+                                                 (128, 3, 128, 100, L.RQ_CODES_PACKED),
+                                                 (64, 2, 128, 64, L.RQ_CODES_INT8),
                                                  (128, 4, 128, 136, L.RQ_CODES_PACKED),
                                                  (256, 2, 256, 129, L.RQ_CODES_PACKED)])
 def test_score_two_stage_shapes(d, bits, m, nq, layout):
@@ -424,7 +435,7 @@ def test_score_two_stage_shapes(d, bits, m, nq, layout):
     ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4 + 1, dtype=torch.float32, device=DEV)
     L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits, layout=layout,
                 use_signs=1, sign_seed=9, centroids=cent)
-    assert L.rq_last_launch() == score_kernels(nq)
+    assert L.rq_last_launch() == score_kernels(nq, d, m, bits, layout)
     torch.cuda.synchronize()
     q16 = u16(q)
     n16 = norms.cpu().numpy().view(np.uint16)

@@ -152,3 +152,27 @@ def test_probe_and_trace_validate_before_any_launch():
         assert L.rq_last_launch() == ""
     assert L.lib().rq_quantize(None, 1, 128, 96, 4, 0, 0, 0, None, None, None, None) == -1
     assert L.rq_last_launch() == ""
+
+
+def test_attention_validates_before_any_launch():
+    """qjl_attention rejects shapes it does not take (RQ_EUNSUPPORTED), an
+    empty key range and a bad scale (RQ_EINVAL), and an undersized workspace
+    (RQ_ESIZE, or the device query without a GPU), all before any launch."""
+    import torch
+    vc = L.rq_lloyd_max(4)
+
+    def call(nq=32, d=128, m=256, T=1000, scale=0.1, ws_numel=1 << 30, kw=None):
+        return L.qjl_attention(FakeTensor(0x40000), 4, nq, d, m, FakeTensor(0x50000), FakeTensor(0x60000),
+                               FakeTensor(0x70000), T, FakeTensor(0x80000), FakeTensor(0x90000), 4, vc,
+                               FakeTensor(0xa0000), FakeTensor(0xb0000, numel=ws_numel), scale, stream=0,
+                               **(kw or {}))
+    for args, status in (((dict(nq=33),), -4), ((dict(d=64),), -4), ((dict(m=136),), -4),
+                         ((dict(T=0),), -1), ((dict(scale=float("nan")),), -1), ((dict(scale=-1.0),), -1)):
+        with pytest.raises(L.RQError) as e:
+            call(**args[0])
+        assert e.value.status == status, (args, e.value.status)
+        assert L.rq_last_launch() == ""
+    if not torch.cuda.is_available():
+        with pytest.raises(L.RQError) as e:
+            call(ws_numel=4)
+        assert e.value.status == -5                           # stops at the device query
