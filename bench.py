@@ -229,7 +229,7 @@ def l2_flusher(dev):
 # current kernels (profiles/quantize_dequantize_llama7b_layer.md): the
 # quantize and dequantize of one Llama-7B-shaped layer (202,375,168 values).
 # Set back to None whenever either kernel changes.
-NCU_DRAM_LAYER = {"quantize": 405_248_512 + 81_866_240, "dequantize": 104_414_976 + 345_299_456}
+NCU_DRAM_LAYER = {"quantize": 405_248_512 + 81_866_240, "dequantize": 104_401_152 + 345_138_944}
 
 
 def run_headline(args, dev, world, rank):
@@ -294,7 +294,7 @@ def run_headline(args, dev, world, rank):
                            alg_bytes_per_launch=alg_quant(LAYER_N), launches_timed=len(q_ms))
     else:
         dom = roofline_hbm(alg_dequant(LAYER_N), mdq, NCU_DRAM_LAYER["dequantize"],
-                           kernel="dequantize_v5_kernel<4,bf16,signs> (d=128)",
+                           kernel="dequantize_v5p_kernel<4,bf16,signs> (d=128)",
                            alg_bytes_per_launch=alg_dequant(LAYER_N), launches_timed=len(dq_ms))
     dom["traffic_note"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch on one layer "
                            "(profiles/); null when not captured for this build")

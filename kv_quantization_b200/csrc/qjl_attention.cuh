@@ -19,9 +19,11 @@
 //
 // Main kernel, per (group, 256-token tile), one CTA per SM over a contiguous
 // range of tiles (queries on M as in qjl_score_v5.cuh):
-//   producers (8 warps, thread = token): key slices as score_v5; the token's
-//     value row as fp16 V' = fp16(c[v_t]) * fp16(n_t / d) into a 128-token
-//     value slice (MN-major B operand: token rows, two 64-wide atoms of d);
+//   key producers (4 warps, thread = tokens r and r + 128): key slices as
+//     score_v5; value producers (4 more warps, the same rows): the value rows
+//     as fp16 V' = fp16(c[v_t]) * fp16(n_t / d) into two 128-token value
+//     slices (MN-major B operand: token rows, two 64-wide atoms of d), so that
+//     the keys of the next tile are unpacked while the values wait for P . V;
 //   MMA issuer 1: S[q][t] = A_q . K_t (M = 128, N = 256) into TMEM;
 //   softmax warps (4 warps of TMEM lane quarter 0: lane = query, 64 columns
 //     each): a = S * g_t * (||q|| scale log2 e) (g_t the score's per-token
@@ -35,7 +37,8 @@
 // ordered (CTA, group) segments).
 //
 // Combine kernel, per (group, query): M = max m_s, L = sum l_s 2^(m_s - M),
-// o = sum O_s 2^(m_s - M) / (2^14 L), then the fp32 radix-2 transform of o
+// o = sum O_s 2^(m_s - M) / L (l and O both carry the factor 2^14 of the
+// weights), then the fp32 radix-2 transform of o
 // (stages h = 1 ... d/2) and the value sign diagonal: out = D H o.
 #pragma once
 #include "qjl_score_v5.cuh"
@@ -51,7 +54,7 @@ constexpr int kAtPBuf = 4 * 32 * 128;            // 4 regions of 64 tokens x 32 
 constexpr int kAtMaxQ = 32;
 constexpr int kAtMaxKRing = 3;
 constexpr int kAtMaxRec = 3;
-constexpr float kAtPScale = 16384.0f;            // P' = 2^14 p keeps small weights normal in fp16
+constexpr float kAtPExp = 14.0f;                 // P' = 2^14 p keeps small weights normal in fp16
 
 __host__ __device__ inline int at_kcopies() { return 8; }
 __host__ __device__ inline size_t at_klut_bytes(bool two, int pw)
@@ -71,7 +74,6 @@ __host__ __device__ inline size_t at_smem(int d, int m, bool two, int pw, int vp
     b += (size_t)2 * kAtVSlice;                                    // value slices
     b += (size_t)2 * kAtPBuf;                                      // P' (double buffer)
     b += (size_t)nrec * ((sc5_rec_bytes(d, m, two, pw) + 127) & ~(size_t)127);   // key records (absorb the P overrun)
-    b += (size_t)256 * 2 * 16;                                     // sign LUT, 2 copies
     b += at_klut_bytes(two, pw) + at_vlut_bytes(vpw);
     b += (size_t)4 * 64 * 4 + 2 * 4 * 32 * 4 + 4 * 32 * 4;         // per-token factors, max and sum exchange
     return b + 8 * (2 * kAtMaxKRing + 2 * 2 + 2 * kAtMaxRec + 2 + 2 * 2 + 2 * 2 + 1) + 16;
@@ -133,8 +135,7 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
     uint8_t *sV = sK + (size_t)kring * kAtKSlice;
     uint8_t *sP = sV + (size_t)2 * kAtVSlice;
     uint8_t *sR = sP + (size_t)2 * kAtPBuf;
-    uint4 *slut = reinterpret_cast<uint4 *>(sR + (size_t)nrec * rec_stride);
-    uint32_t *klut = reinterpret_cast<uint32_t *>(slut + 256 * 2);
+    uint32_t *klut = reinterpret_cast<uint32_t *>(sR + (size_t)nrec * rec_stride);
     uint32_t *vlut = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(klut) + at_klut_bytes(TWO, PW));
     float *sG = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(vlut) + at_vlut_bytes(VPW));   // [4][64]
     float *sXM = sG + 4 * 64;                                       // [2][4][32] tile maxima
@@ -155,17 +156,6 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int i = tid; i < 256 * 2; i += kAtThreads) {
-        const int byte = i >> 1;
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t lo = ((byte >> (2 * k)) & 1) ? 0x3C00u : 0xBC00u;
-            const uint32_t hi = ((byte >> (2 * k + 1)) & 1) ? 0x3C00u : 0xBC00u;
-            w[k] = lo | (hi << 16);
-        }
-        slut[i] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
     // centroid pair tables (fp16), 8 copies (lane % 8)
     auto fill_pairs = [&](const QuantTables &T, uint32_t *lut, int pw) {
         if (pw <= 4) {
@@ -186,9 +176,9 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
     if (TWO) fill_pairs(TK, klut, PW);
     fill_pairs(TV, vlut, VPW);
     if (tid == 0) {
-        for (int b = 0; b < kring; ++b) { mbar_init(&k_full[b], 8); mbar_init(&k_empty[b], 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(&v_full[b], 4); mbar_init(&v_empty[b], 1); }
-        for (int r = 0; r < nrec; ++r) { mbar_init(&r_full[r], 1); mbar_init(&r_empty[r], 8); }
+        for (int b = 0; b < kring; ++b) { mbar_init(&k_full[b], 4); mbar_init(&k_empty[b], 1); }   // 4 key producer warps
+        for (int b = 0; b < 2; ++b) { mbar_init(&v_full[b], 4); mbar_init(&v_empty[b], 1); }       // 4 value producer warps
+        for (int r = 0; r < nrec; ++r) { mbar_init(&r_full[r], 1); mbar_init(&r_empty[r], 4); }
         mbar_init(s_full, 1);
         mbar_init(s_empty, 4);
         for (int b = 0; b < 2; ++b) {
@@ -228,90 +218,75 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
                 if (TWO) bulk_load(R + (size_t)kAtTok * sbytes, codes + (g * T_len + t0) * cbytes, cb, &r_full[rs]);
             }
         }
-    } else if (pidx >= 0) {
-        // ------------------------------------------------------------ producers (thread = token row)
-        const int r = pidx * 32 + lane;                           // 0..255
-        const int vh = r >> 7, vr = r & 127;                      // value slice (tile half) and row in it
+    } else if (pidx >= 0 && pidx < 4) {
+        // ------------------------------------------------------------ key producers (thread = rows r, r + 128)
         const float kq = 1.2533141373155002512f / (float)m;
-        const uint32_t lane8 = (uint32_t)(lane & 7), lane2 = (uint32_t)(lane & 1);
+        const uint32_t lane8 = (uint32_t)(lane & 7);
         int64_t slice = 0;
         for (int64_t it = it0; it < it1 && ok; ++it) {
             const int64_t k = it - it0;
             const int rs = (int)(k % nrec);
             const int64_t g = it / tiles_per_g, t0 = (it % tiles_per_g) * kAtTok;
-            const bool tv = t0 + r < T_len;
-            const int64_t kt = g * T_len + t0 + r;
-            // the value row's codes and norm (loaded early, used after the keys)
-            uint4 vc[vcb / 16];
-            uint32_t vf2 = 0u;
-#pragma unroll
-            for (int i = 0; i < (int)(vcb / 16); ++i)
-                vc[i] = tv ? __ldg(reinterpret_cast<const uint4 *>(vcodes + kt * vcb) + i) : make_uint4(0u, 0u, 0u, 0u);
-            if (tv) {
-                const float fv = __fmul_rn(h16_to_f32(__ldg(vnorms + kt)), 1.0f / (float)kAtD);
-                const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(fv));
-                vf2 = h | (h << 16);
-            }
-            uint32_t rho2 = 0x3C003C00u;
+            uint32_t rho2[2] = {0x3C003C00u, 0x3C003C00u};
             if (TWO) {
-                float rho = 0.0f;
-                if (tv) {
-                    const float n1 = h16_to_f32(__ldg(norms + kt));
-                    const float rn = h16_to_f32(__ldg(sk_norms + kt));
-                    if (n1 > 0.0f) rho = __fdiv_rn(__fmul_rn(__fmul_rn(kq, rn), (float)d), n1);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = pidx * 32 + lane + 128 * h;
+                    float rho = 0.0f;
+                    if (t0 + r < T_len) {
+                        const int64_t kt = g * T_len + t0 + r;
+                        const float n1 = h16_to_f32(__ldg(norms + kt));
+                        const float rn = h16_to_f32(__ldg(sk_norms + kt));
+                        if (n1 > 0.0f) rho = __fdiv_rn(__fmul_rn(__fmul_rn(kq, rn), (float)d), n1);
+                    }
+                    const uint32_t hh = (uint32_t)__half_as_ushort(__float2half_rn(rho));
+                    rho2[h] = hh | (hh << 16);
                 }
-                const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(rho));
-                rho2 = h | (h << 16);
             }
             if (ok && !mbar_wait(&r_full[rs], (uint32_t)((k / nrec) & 1))) ok = false;
             const uint8_t *R = sR + (size_t)rs * rec_stride;
-            const uint8_t *Rs = R + (size_t)r * sbytes;
-            const uint8_t *Rc = R + (size_t)kAtTok * sbytes + (size_t)r * cbytes;
             for (int s = 0; s < nsl; ++s, ++slice) {
                 const int b = (int)(slice % kring);
                 const int64_t use = slice / kring;
                 if (use > 0 && ok && !mbar_wait(&k_empty[b], (uint32_t)((use - 1) & 1))) ok = false;
-                uint8_t *Br = sK + (size_t)b * kAtKSlice + (size_t)(r >> 3) * 1024 + (size_t)(r & 7) * 128;
-                if (TWO && s < dsl) {
-                    uint32_t cw[2 * PW];
-                    const uint8_t *cp = Rc + s * 8 * PW;
 #pragma unroll
-                    for (int q = 0; q < PW; ++q) {
-                        const uint2 v2 = *reinterpret_cast<const uint2 *>(cp + 8 * q);
-                        cw[2 * q] = v2.x;
-                        cw[2 * q + 1] = v2.y;
-                    }
+                for (int h = 0; h < 2; ++h) {
+                    const int r = pidx * 32 + lane + 128 * h;
+                    uint8_t *Br = sK + (size_t)b * kAtKSlice + (size_t)(r >> 3) * 1024 + (size_t)(r & 7) * 128;
+                    if (TWO && s < dsl) {
+                        uint32_t cw[2 * PW];
+                        const uint8_t *cp = R + (size_t)kAtTok * sbytes + (size_t)r * cbytes + s * 8 * PW;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        uint32_t o[4];
+                        for (int q = 0; q < PW; ++q) {
+                            const uint2 v2 = *reinterpret_cast<const uint2 *>(cp + 8 * q);
+                            cw[2 * q] = v2.x;
+                            cw[2 * q + 1] = v2.y;
+                        }
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const uint32_t ca = unpack_code<64, PW>(cw, 8 * kk + 2 * e);
-                            const uint32_t cb2 = unpack_code<64, PW>(cw, 8 * kk + 2 * e + 1);
-                            if constexpr (PW <= 4) {
-                                o[e] = klut[((ca | (cb2 << PW)) << 3) + lane8];
-                            } else {
-                                const uint16_t *k16 = reinterpret_cast<const uint16_t *>(klut);
-                                o[e] = (uint32_t)k16[(ca << 3) + lane8] | ((uint32_t)k16[(cb2 << 3) + lane8] << 16);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            uint32_t o[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t ca = unpack_code<64, PW>(cw, 8 * kk + 2 * e);
+                                const uint32_t cb2 = unpack_code<64, PW>(cw, 8 * kk + 2 * e + 1);
+                                if constexpr (PW <= 4) {
+                                    o[e] = klut[((ca | (cb2 << PW)) << 3) + lane8];
+                                } else {
+                                    const uint16_t *k16 = reinterpret_cast<const uint16_t *>(klut);
+                                    o[e] = (uint32_t)k16[(ca << 3) + lane8] | ((uint32_t)k16[(cb2 << 3) + lane8] << 16);
+                                }
                             }
+                            *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                         }
-                        *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                } else {
-                    const int sc0 = (s - dsl) * 64;
-                    const uint2 v2 = *reinterpret_cast<const uint2 *>(Rs + sc0 / 8);
-                    const uint32_t sb[2] = {v2.x, v2.y};
+                    } else {
+                        const int sc0 = (s - dsl) * 64;
+                        const uint2 v2 = *reinterpret_cast<const uint2 *>(R + (size_t)r * sbytes + sc0 / 8);
+                        const uint32_t sb[2] = {v2.x, v2.y};
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t byte = (sb[kk >> 2] >> (8 * (kk & 3))) & 0xffu;
-                        uint4 v = slut[(byte << 1) + lane2];
-                        if (TWO) {
-                            v.x = (v.x & 0x80008000u) | rho2;
-                            v.y = (v.y & 0x80008000u) | rho2;
-                            v.z = (v.z & 0x80008000u) | rho2;
-                            v.w = (v.w & 0x80008000u) | rho2;
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t byte = (sb[kk >> 2] >> (8 * (kk & 3))) & 0xffu;
+                            *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = signs8_to_h2x4(byte, rho2[h]);
                         }
-                        *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = v;
                     }
                 }
                 fence_proxy_async_smem();
@@ -320,39 +295,59 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&r_empty[rs]);
-            // value row: V' = fp16(c) * fp16(n / d), rows of the MN-major B operand (two 64-wide atoms of d)
-            if (k > 0 && ok && !mbar_wait(&v_empty[vh], (uint32_t)((k - 1) & 1))) ok = false;
-            uint8_t *Vr = sV + (size_t)vh * kAtVSlice + (size_t)(vr >> 3) * 1024 + (size_t)(vr & 7) * 128;
-            uint32_t vw[vcb / 4];
+        }
+    } else if (pidx >= 4) {
+        // ------------------------------------------------------------ value producers (thread = rows r, r + 128)
+        const uint32_t lane8 = (uint32_t)(lane & 7);
+        const int vr = (pidx - 4) * 32 + lane;                   // row in each 128-token value slice
+        for (int64_t it = it0; it < it1 && ok; ++it) {
+            const int64_t k = it - it0;
+            const int64_t g = it / tiles_per_g, t0 = (it % tiles_per_g) * kAtTok;
+#pragma unroll 1
+            for (int vh = 0; vh < 2; ++vh) {
+                const int r = vh * 128 + vr;
+                const bool tv = t0 + r < T_len;
+                const int64_t kt = g * T_len + t0 + r;
+                uint32_t vw[vcb / 4];
+                uint32_t vf2 = 0u;
 #pragma unroll
-            for (int i = 0; i < (int)(vcb / 16); ++i) {
-                vw[4 * i] = vc[i].x; vw[4 * i + 1] = vc[i].y; vw[4 * i + 2] = vc[i].z; vw[4 * i + 3] = vc[i].w;
-            }
-#pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {                     // 16 chunks of 8 values: d = 8 ch ... 8 ch + 7
-                uint32_t o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 8 * ch + 2 * e;
-                    const uint32_t ca = unpack_code<kAtD, VPW>(vw, j), cb2 = unpack_code<kAtD, VPW>(vw, j + 1);
-                    uint32_t pr;
-                    if constexpr (VPW <= 4) {
-                        pr = vlut[((ca | (cb2 << VPW)) << 3) + lane8];
-                    } else {
-                        const uint16_t *v16 = reinterpret_cast<const uint16_t *>(vlut);
-                        pr = (uint32_t)v16[(ca << 3) + lane8] | ((uint32_t)v16[(cb2 << 3) + lane8] << 16);
-                    }
-                    const __half2 hv = __hmul2(*reinterpret_cast<const __half2 *>(&pr),
-                                               *reinterpret_cast<const __half2 *>(&vf2));
-                    o[e] = tv ? *reinterpret_cast<const uint32_t *>(&hv) : 0u;
+                for (int i = 0; i < (int)(vcb / 16); ++i) {
+                    const uint4 v4 = tv ? __ldg(reinterpret_cast<const uint4 *>(vcodes + kt * vcb) + i) : make_uint4(0u, 0u, 0u, 0u);
+                    vw[4 * i] = v4.x; vw[4 * i + 1] = v4.y; vw[4 * i + 2] = v4.z; vw[4 * i + 3] = v4.w;
                 }
-                const int atom = ch >> 3, c8 = ch & 7;
-                *reinterpret_cast<uint4 *>(Vr + (size_t)atom * (kAtVSlice / 2) + ((c8 ^ (vr & 7)) << 4)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
+                if (tv) {
+                    const float fv = __fmul_rn(h16_to_f32(__ldg(vnorms + kt)), 1.0f / (float)kAtD);
+                    const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(fv));
+                    vf2 = h | (h << 16);
+                }
+                if (k > 0 && ok && !mbar_wait(&v_empty[vh], (uint32_t)((k - 1) & 1))) ok = false;
+                uint8_t *Vr = sV + (size_t)vh * kAtVSlice + (size_t)(vr >> 3) * 1024 + (size_t)(vr & 7) * 128;
+#pragma unroll
+                for (int ch = 0; ch < 16; ++ch) {                 // 16 chunks of 8 values: d = 8 ch ... 8 ch + 7
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 8 * ch + 2 * e;
+                        const uint32_t ca = unpack_code<kAtD, VPW>(vw, j), cb2 = unpack_code<kAtD, VPW>(vw, j + 1);
+                        uint32_t pr;
+                        if constexpr (VPW <= 4) {
+                            pr = vlut[((ca | (cb2 << VPW)) << 3) + lane8];
+                        } else {
+                            const uint16_t *v16 = reinterpret_cast<const uint16_t *>(vlut);
+                            pr = (uint32_t)v16[(ca << 3) + lane8] | ((uint32_t)v16[(cb2 << 3) + lane8] << 16);
+                        }
+                        const __half2 hv = __hmul2(*reinterpret_cast<const __half2 *>(&pr),
+                                                   *reinterpret_cast<const __half2 *>(&vf2));
+                        o[e] = tv ? *reinterpret_cast<const uint32_t *>(&hv) : 0u;
+                    }
+                    const int atom = ch >> 3, c8 = ch & 7;
+                    *reinterpret_cast<uint4 *>(Vr + (size_t)atom * (kAtVSlice / 2) + ((c8 ^ (vr & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&v_full[vh]);
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&v_full[vh]);
         }
     } else if (warp == 11) {
         // ------------------------------------------------------------ MMA 1: S = A_q . K
@@ -451,6 +446,13 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
 #pragma unroll
         for (int j = 0; j < 32; ++j) O[j] = 0.0f;
         int64_t pending = -1;                                    // tile whose O_tile is still to be folded in
+        float gn0 = 0.0f, gn1 = 0.0f;                            // norms of this lane's two columns, next tile
+        auto load_g = [&](int64_t it) {
+            const int64_t g = it / tiles_per_g, ta = (it % tiles_per_g) * kAtTok + kw * 64 + 2 * lane;
+            gn0 = ta < T_len ? h16_to_f32(__ldg(gsrc + g * T_len + ta)) : 0.0f;
+            gn1 = ta + 1 < T_len ? h16_to_f32(__ldg(gsrc + g * T_len + ta + 1)) : 0.0f;
+        };
+        if (it0 < it1) load_g(it0);
         auto fold = [&](int64_t c, float alpha) {
             const int b = (int)(c & 1);
             if (ok && !mbar_wait(&o_full[b], (uint32_t)((c >> 1) & 1))) ok = false;
@@ -473,17 +475,12 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
             const int64_t g = it / tiles_per_g, t0 = (it % tiles_per_g) * kAtTok;
             const bool seg_start = it == it0 || (it - 1) / tiles_per_g != g;
             if (seg_start) cq = qi < nq ? __fmul_rn(__ldg(wsN + g * nq + qi), qscale) : 0.0f;
-            // per-token score factors of this warp's 64 columns
+            // per-token score factors of this warp's 64 columns (loaded one tile ahead)
             __syncwarp();                                        // the previous tile's reads of gw are done
-            {
-                const int64_t ta = t0 + kw * 64 + 2 * lane;
-                const float n0 = ta < T_len ? h16_to_f32(__ldg(gsrc + g * T_len + ta)) : 0.0f;
-                const float n1 = ta + 1 < T_len ? h16_to_f32(__ldg(gsrc + g * T_len + ta + 1)) : 0.0f;
-                const float f0 = TWO ? __fmul_rn(n0, inv_d) : __fmul_rn(kq, n0);
-                const float f1 = TWO ? __fmul_rn(n1, inv_d) : __fmul_rn(kq, n1);
-                *reinterpret_cast<float2 *>(gw + 2 * lane) = make_float2(f0, f1);
-            }
+            *reinterpret_cast<float2 *>(gw + 2 * lane) = make_float2(TWO ? __fmul_rn(gn0, inv_d) : __fmul_rn(kq, gn0),
+                                                                     TWO ? __fmul_rn(gn1, inv_d) : __fmul_rn(kq, gn1));
             __syncwarp();
+            if (it + 1 < it1) load_g(it + 1);
             if (ok && !mbar_wait(s_full, (uint32_t)(c & 1))) ok = false;
             tc_fence_after();
             uint32_t sr[64];
@@ -495,12 +492,17 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
             if (lane == 0) mbar_arrive(s_empty);
             const int64_t tcol = t0 + kw * 64;                   // token of column 0 of this warp
             const int nvalid = T_len - tcol >= 64 ? 64 : (T_len - tcol > 0 ? (int)(T_len - tcol) : 0);
-            // a_j = S_j g_j ||q|| scale log2(e), computed twice (max, then exp) to keep registers low
+            // a_j = S_j g_j ||q|| scale log2(e), kept in place of S_j
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float v = __fmul_rn(__fmul_rn(__uint_as_float(sr[j]), gw[j]), cq);
-                if (j < nvalid) mx = fmaxf(mx, v);
+            for (int j = 0; j < 64; j += 2) {
+                const float2 gj = *reinterpret_cast<const float2 *>(gw + j);
+                const float2 v = __fmul2_rn(__fmul2_rn(make_float2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), gj),
+                                            make_float2(cq, cq));
+                sr[j] = __float_as_uint(v.x);
+                sr[j + 1] = __float_as_uint(v.y);
+                if (j < nvalid) mx = fmaxf(mx, v.x);
+                if (j + 1 < nvalid) mx = fmaxf(mx, v.y);
             }
             float *xm = sXM + (c & 1) * 128;
             xm[kw * 32 + lane] = mx;
@@ -508,9 +510,10 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
             const float mt = fmaxf(fmaxf(xm[lane], xm[32 + lane]), fmaxf(xm[64 + lane], xm[96 + lane]));
             const float mnew = fmaxf(mrun, mt);
             const float alpha = ex2_approx(mrun - mnew);        // 0 for the first tile (mrun = -inf)
-            // P' row (query qi) of tokens 64 kw ... 64 kw + 63: region kw of buffer b
+            // P' = 2^14 p = 2^(a - m + 14): row qi of tokens 64 kw ... 64 kw + 63, region kw of buffer b
             if (c >= 2 && ok && !mbar_wait(&p_empty[b], (uint32_t)(((c >> 1) - 1) & 1))) ok = false;
             uint8_t *Pr = sP + (size_t)b * kAtPBuf + (size_t)kw * 4096 + (size_t)(qi >> 3) * 1024 + (size_t)(qi & 7) * 128;
+            const float moff = mnew - kAtPExp;
             float ls = 0.0f;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
@@ -518,12 +521,10 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = 8 * ch + 2 * e;
-                    const float v0 = __fmul_rn(__fmul_rn(__uint_as_float(sr[j]), gw[j]), cq);
-                    const float v1 = __fmul_rn(__fmul_rn(__uint_as_float(sr[j + 1]), gw[j + 1]), cq);
-                    const float p0 = j < nvalid ? ex2_approx(v0 - mnew) : 0.0f;
-                    const float p1 = j + 1 < nvalid ? ex2_approx(v1 - mnew) : 0.0f;
+                    const float p0 = j < nvalid ? ex2_approx(__uint_as_float(sr[j]) - moff) : 0.0f;
+                    const float p1 = j + 1 < nvalid ? ex2_approx(__uint_as_float(sr[j + 1]) - moff) : 0.0f;
                     ls += p0 + p1;
-                    const __half2 h = __floats2half2_rn(__fmul_rn(p0, kAtPScale), __fmul_rn(p1, kAtPScale));
+                    const __half2 h = __floats2half2_rn(p0, p1);
                     w4[e] = *reinterpret_cast<const uint32_t *>(&h);
                 }
                 *reinterpret_cast<uint4 *>(Pr + ((ch ^ (qi & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -599,7 +600,7 @@ attention_combine_kernel(const float *__restrict__ part, int nq, int d, int64_t 
         L = __fmaf_rn(P[(size_t)nq * d + nq + qi], w, L);
         acc = __fmaf_rn(P[(size_t)qi * d + j], w, acc);
     }
-    o[j] = acc / (L * kAtPScale);
+    o[j] = acc / L;                                  // O and l both carry the factor 2^14
     __syncthreads();
     for (int h = 1; h < d; h *= 2) {
         float v = 0.0f;

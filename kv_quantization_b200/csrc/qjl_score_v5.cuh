@@ -6,11 +6,13 @@
 // to fp16 (centroid values for the first-stage codes, signs for the sketch),
 // and the score is the fp32 dot product times per-token and per-query
 // factors.  The operands are swapped: D[q][t] = A[q] . B[t] with
-//   A = the group's queries, M = 128 rows (rows >= n_q are not read back),
+//   A = the group's queries, M = 64 (n_q <= 64) or 128 rows (rows >= n_q are
+//   not read back),
 //   B = 256 key tokens, N = 256,
-// because one tcgen05.mma kind::f16 instruction (K = 16) occupies the tensor
-// pipe for about 142 cycles whatever its N from 32 to 256 (measured on B200):
-// a 256-token instruction does eight times the work of a 32-query one.
+// because a thread issuing tcgen05.mma kind::f16 (K = 16) gets one
+// instruction through about every 150 cycles whatever its M and N (measured
+// on B200): a 256-token instruction does eight times the work of a 32-query
+// one in the same issue time.
 //
 // Per-token factors.  Pure QJL: score = ||q|| * (kq * rn_t) * D[q][t] with
 // B = +-1, kq = sqrt(pi/2) / m.  Two-stage keys: the sign columns of B carry
@@ -28,9 +30,13 @@
 //   warp 17 (MMA)      : per slice four MMAs into one of two 256-column TMEM
 //                        accumulators; reloads the group's queries (A) when
 //                        the group changes, after its MMAs have drained;
-//   warps 8-15 (epilogue): warp w reads TMEM lanes 32 (w % 4) ... (queries)
+//   warps 8-15 (epilogue): warp w reads TMEM lane quarter w % 4 (queries)
 //                        and columns 128 ((w - 8) / 4) ... of the tile, scales
-//                        and stores 16-byte runs of scores[g][q][t].
+//                        them (per-token factors loaded one tile ahead) and
+//                        stores 16-byte runs of scores[g][q][t].
+// With n_q <= 64 the MMAs are M = 64: half the A operand is read per
+// instruction, and the 64 rows spread over the four lane quarters (16 each),
+// so that up to four quarters' epilogue warps share the output.
 #pragma once
 #include "qjl_score_v4.cuh"
 
@@ -43,6 +49,7 @@ constexpr int kSc5MaxRing = 6;
 constexpr int kSc5MaxRec = 4;
 
 __host__ __device__ inline int sc5_qrows(int nq) { return (nq + 7) & ~7; }
+
 // A: one 64-column region of qrows rows per slice; the MMA reads 128 rows, the
 // rows past qrows fall on whatever follows (never read back).
 __host__ __device__ inline size_t sc5_a_bytes(int nq, int kb)
@@ -60,7 +67,6 @@ __host__ __device__ inline size_t sc5_smem(int nq, int d, int m, bool two, int p
     b += (sc5_a_bytes(nq, kb) + 1023) & ~(size_t)1023;            // A (queries)
     b += (size_t)ring * kSc5SliceBytes;                            // B ring (also absorbs the A overrun)
     b += (size_t)nrec * ((sc5_rec_bytes(d, m, two, pw) + 127) & ~(size_t)127);   // records
-    b += (size_t)256 * 8 * 16;                                     // sign LUT, 8 copies
     if (two) b += pw <= 4 ? ((size_t)1 << (2 * pw)) * 32 * 4 : ((size_t)1 << pw) * 32 * 2;
     b += (size_t)8 * 128 * 4;                                      // epilogue per-token factors
     return b + 8 * (2 * kSc5MaxRing + 2 * kSc5MaxRec + 5) + 16;
@@ -73,6 +79,21 @@ __host__ __device__ inline bool sc5_eligible(int nq, int d, int m, bool two, int
     if ((m / 8) % 16 != 0) return false;                 // sign bytes of a token: a multiple of 16
     if (two && (d * pw / 8) % 16 != 0) return false;     // code bytes of a token: a multiple of 16
     return true;
+}
+
+// Eight sign bits -> eight fp16 values +-mag (bit 1 -> +mag): mag2 holds the
+// magnitude in both halves, the sign of value 2k (2k + 1) goes to bit 15 (31)
+// of word k.  ALU only, so the shared-memory bandwidth stays with the
+// tensor-core operands.
+__device__ __forceinline__ uint4 signs8_to_h2x4(uint32_t byte, uint32_t mag2)
+{
+    const uint32_t nb = ~byte;
+    uint4 v;
+    v.x = mag2 | ((nb << 15) & 0x00008000u) | ((nb << 30) & 0x80000000u);
+    v.y = mag2 | ((nb << 13) & 0x00008000u) | ((nb << 28) & 0x80000000u);
+    v.z = mag2 | ((nb << 11) & 0x00008000u) | ((nb << 26) & 0x80000000u);
+    v.w = mag2 | ((nb << 9) & 0x00008000u) | ((nb << 24) & 0x80000000u);
+    return v;
 }
 
 template <int PW, bool TWO>
@@ -94,8 +115,7 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
     uint8_t *sA = base;
     uint8_t *sB = sA + ((sc5_a_bytes(nq, kb) + 1023) & ~(size_t)1023);
     uint8_t *sR = sB + (size_t)ring * kSc5SliceBytes;
-    uint4 *slut = reinterpret_cast<uint4 *>(sR + (size_t)nrec * rec_stride);
-    uint32_t *clut = reinterpret_cast<uint32_t *>(slut + 256 * 8);
+    uint32_t *clut = reinterpret_cast<uint32_t *>(sR + (size_t)nrec * rec_stride);
     const size_t clut_bytes = TWO ? (PW <= 4 ? ((size_t)1 << (2 * PW)) * 32 * 4 : ((size_t)1 << PW) * 32 * 2) : 0;
     float *sF = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(clut) + clut_bytes);
     uint64_t *b_full = reinterpret_cast<uint64_t *>(sF + 8 * 128);
@@ -108,18 +128,6 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // byte -> eight fp16 +-1 (bit 1 -> +1), eight copies (lane % 8)
-    for (int i = tid; i < 256 * 8; i += kSc5Threads) {
-        const int byte = i >> 3;
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t lo = ((byte >> (2 * k)) & 1) ? 0x3C00u : 0xBC00u;
-            const uint32_t hi = ((byte >> (2 * k + 1)) & 1) ? 0x3C00u : 0xBC00u;
-            w[k] = lo | (hi << 16);
-        }
-        slut[i] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
     if constexpr (TWO) {
         if constexpr (PW <= 4) {
             for (int i = tid; i < (1 << (2 * PW)) * 32; i += kSc5Threads) {
@@ -184,7 +192,6 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
         // ------------------------------------------------------------ producers
         const int r = tid;                           // token row of the tile, 0..255
         const float kq = 1.2533141373155002512f / (float)m;
-        const uint32_t lut_lane = (uint32_t)(lane & 7);
         int64_t slice = 0;
         for (int64_t it = it0; it < it1 && ok; ++it) {
             const int64_t k = it - it0;
@@ -243,15 +250,7 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t byte = (sb[kk >> 2] >> (8 * (kk & 3))) & 0xffu;
-                        uint4 v = slut[(byte << 3) + lut_lane];
-                        if (TWO) {
-                            // +-1 -> +-rho: keep each half's sign, take rho's magnitude
-                            v.x = (v.x & 0x80008000u) | rho2;
-                            v.y = (v.y & 0x80008000u) | rho2;
-                            v.z = (v.z & 0x80008000u) | rho2;
-                            v.w = (v.w & 0x80008000u) | rho2;
-                        }
-                        *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = v;
+                        *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = signs8_to_h2x4(byte, rho2);
                     }
                 }
                 fence_proxy_async_smem();
@@ -264,7 +263,7 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
     } else if (warp == 17) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
-        const uint32_t idesc = idesc_f16(false, 128, kSc5Tok);
+        const uint32_t idesc = idesc_f16(false, nq <= 64 ? 64 : 128, kSc5Tok);
         const uint32_t aregion = (uint32_t)qrows * 128u;
         int64_t cur_g = -1, slice = 0;
         uint32_t done_phase = 0;
@@ -317,33 +316,44 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
         }
     } else {
         // ------------------------------------------------------------ epilogue (warps 8-15)
+        // M = 64 accumulators (n_q <= 64) keep row r in TMEM lane 32 (r / 16) + r % 16; M = 128
+        // ones keep row r in lane r.
         const int quarter = warp & 3;
         const int half = (warp - 8) >> 2;
-        const int qi = quarter * 32 + lane;                 // query row of this thread
-        const bool live = quarter * 32 < nq;                // this warp's lanes hold queries at all
+        const bool m64 = nq <= 64;
+        const int qi = m64 ? quarter * 16 + lane : quarter * 32 + lane;     // query row of this thread
+        const bool lane_ok = (m64 ? lane < 16 : true) && qi < nq;
+        const bool live = (m64 ? quarter * 16 : quarter * 32) < nq;         // the warp has queries at all
         const float kq = 1.2533141373155002512f / (float)m;
         const float inv_d = 1.0f / (float)d;
         const uint16_t *nsrc = TWO ? norms : sk_norms;
         float *fac = sF + (warp - 8) * 128;                 // this warp's per-token factors
         int64_t qn_g = -1;
         float qn = 0.0f;
+        // lane l holds the factors of tokens 4 l ... 4 l + 3 of the warp's 128 columns; the next
+        // tile's are loaded while this one is processed
+        auto load_f = [&](int64_t it, float *f) {
+            const int64_t g = it / tiles_per_g, tb = (it % tiles_per_g) * kSc5Tok + half * 128;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int64_t t = tb + 4 * lane + e;
+                const float nv = t < T_len ? h16_to_f32(__ldg(nsrc + g * T_len + t)) : 0.0f;
+                f[e] = TWO ? __fmul_rn(nv, inv_d) : __fmul_rn(kq, nv);
+            }
+        };
+        float fn[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (live && it0 < it1) load_f(it0, fn);
         for (int64_t it = it0; it < it1 && ok; ++it) {
             const int64_t g = it / tiles_per_g, t0 = (it % tiles_per_g) * kSc5Tok;
             const int a = (int)((it - it0) & 1);
             const int64_t ause = (it - it0) >> 1;
             const int64_t tb = t0 + half * 128;              // first token of this warp's 128 columns
-            float f4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const float f4[4] = {fn[0], fn[1], fn[2], fn[3]};
             if (live) {
+                if (it + 1 < it1) load_f(it + 1, fn);
                 if (g != qn_g) {
-                    qn = qi < nq ? __ldg(wsN + g * nq + qi) : 0.0f;
+                    qn = lane_ok ? __ldg(wsN + g * nq + qi) : 0.0f;
                     qn_g = g;
-                }
-                // lane l: the norms of tokens tb + 4 l ... tb + 4 l + 3 (loaded before the wait)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int64_t t = tb + 4 * lane + e;
-                    const float nv = t < T_len ? h16_to_f32(__ldg(nsrc + g * T_len + t)) : 0.0f;
-                    f4[e] = TWO ? __fmul_rn(nv, inv_d) : __fmul_rn(kq, nv);
                 }
             }
             if (ok && !mbar_wait(&acc_full[a], (uint32_t)(ause & 1))) ok = false;
@@ -351,14 +361,15 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
             if (live && ok) {
                 *reinterpret_cast<float4 *>(fac + 4 * lane) = make_float4(f4[0], f4[1], f4[2], f4[3]);
                 __syncwarp();
+                float *dst0 = scores + ((int64_t)g * nq + qi) * T_len;
                 for (int c = 0; c < 4; ++c) {
                     uint32_t rr[32];
                     tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * kSc5Tok + half * 128 + c * 32),
                               rr);
                     tmem_ld_wait();
                     const int64_t tc0 = tb + c * 32;
-                    if (qi < nq) {
-                        float *dst = scores + ((int64_t)g * nq + qi) * T_len + tc0;
+                    if (lane_ok) {
+                        float *dst = dst0 + tc0;
                         const bool full = tc0 + 32 <= T_len && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
 #pragma unroll
                         for (int i = 0; i < 32; i += 4) {

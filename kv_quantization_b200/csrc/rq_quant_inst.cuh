@@ -207,7 +207,7 @@ static cudaError_t launch_dq5(const DequantArgs &a, cudaStream_t st)
         if (!a.has_tmap_out32) return cudaErrorNotSupported;
         const bool signs = a.tables->sign_words[0] | a.tables->sign_words[1] | a.tables->sign_words[2] |
                            a.tables->sign_words[3];
-        if constexpr (PW <= 3) {                    // pair layout (rq_v5.cuh): measured faster up to 3 bits only
+        if constexpr (PW <= 4) {                    // pair layout (rq_v5.cuh): measured faster up to 4 bits
             const size_t smemp = dequantize_v5p_smem(PW);
             if (smemp <= kMaxSmemPerBlock && a.tables->levels == (1 << PW)) {
                 auto kp = signs ? dequantize_v5p_kernel<PW, BF16, true> : dequantize_v5p_kernel<PW, BF16, false>;

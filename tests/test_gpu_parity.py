@@ -54,11 +54,11 @@ def quant_kernels(d, bits, layout):
     """Kernels the dispatch picks for rq_quantize / rq_dequantize: the d = 128
     one-block-per-thread kernels when a saturating search grid of at most 128
     cells exists (the Lloyd-Max tables of 1-5 bits), the general-d kernels
-    otherwise; 1-3-bit packed d = 128 codes take the pair-table dequantize."""
+    otherwise; 1-4-bit packed d = 128 codes take the pair-table dequantize."""
     q = "quantize_v5_kernel" if d == 128 and bits <= 5 else "quantize_v2_kernel"
     if d != 128:
         dq = "dequantize_v2_kernel"
-    elif layout == L.RQ_CODES_PACKED and bits <= 3:
+    elif layout == L.RQ_CODES_PACKED and bits <= 4:
         dq = "dequantize_v5p_kernel"
     else:
         dq = "dequantize_v5_kernel"
