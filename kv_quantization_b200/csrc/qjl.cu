@@ -207,15 +207,16 @@ static cudaError_t launch_score_v2(const ScoreArgs &a, cudaStream_t st)
         const Cfg5 cfgs5[] = {{4, 3}, {4, 2}, {3, 2}, {2, 2}, {2, 1}};
         const int64_t items5 = a.G * ((a.T + kSc5Tok - 1) / kSc5Tok);
         const int64_t grid5 = items5 < (int64_t)a.num_sms ? items5 : (int64_t)a.num_sms;
+        const bool tma = a.has_tmap_scores && a.nq <= 64;
         for (const Cfg5 &c : cfgs5) {
-            const size_t smem5 = sc5_smem(a.nq, a.d, a.m, TWO, PW, c.ring, c.nrec);
+            const size_t smem5 = sc5_smem(a.nq, a.d, a.m, TWO, PW, c.ring, c.nrec, tma);
             if (smem5 > kMaxSmemPerBlock) continue;
             auto kern5 = score_v5_kernel<PW, TWO>;
             e = cudaFuncSetAttribute(kern5, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem5);
             if (e != cudaSuccess) return e;
             kern5<<<(unsigned)(grid5 > 0 ? grid5 : 1), kSc5Threads, smem5, st>>>(
                 wsB, wsN, a.nq, a.d, a.m, a.signs, a.sk_norms, a.T, a.G, a.codes, a.norms, *a.tables, a.scores,
-                c.ring, c.nrec);
+                c.ring, c.nrec, a.tmap_scores, tma ? 1 : 0);
             note_launch("score_v5_kernel");
             return cudaGetLastError();
         }

@@ -19,11 +19,11 @@
 //
 // Main kernel, per (group, 256-token tile), one CTA per SM over a contiguous
 // range of tiles (queries on M as in qjl_score_v5.cuh):
-//   key producers (4 warps, thread = tokens r and r + 128): key slices as
-//     score_v5; value producers (4 more warps, the same rows): the value rows
-//     as fp16 V' = fp16(c[v_t]) * fp16(n_t / d) into two 128-token value
-//     slices (MN-major B operand: token rows, two 64-wide atoms of d), so that
-//     the keys of the next tile are unpacked while the values wait for P . V;
+//   producers (8 warps, thread = token): key slices as score_v5; then the
+//     token's value row as fp16 V' = fp16(c[v_t]) * fp16(n_t / d) into a
+//     128-token value slice (MN-major B operand: token rows, two 64-wide
+//     atoms of d).  Measured: splitting the warps into key and value groups
+//     made the key unpack (4 warps) the critical path, so all eight do both;
 //   MMA issuer 1: S[q][t] = A_q . K_t (M = 128, N = 256) into TMEM;
 //   softmax warps (4 warps of TMEM lane quarter 0: lane = query, 64 columns
 //     each): a = S * g_t * (||q|| scale log2 e) (g_t the score's per-token
@@ -176,9 +176,9 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
     if (TWO) fill_pairs(TK, klut, PW);
     fill_pairs(TV, vlut, VPW);
     if (tid == 0) {
-        for (int b = 0; b < kring; ++b) { mbar_init(&k_full[b], 4); mbar_init(&k_empty[b], 1); }   // 4 key producer warps
-        for (int b = 0; b < 2; ++b) { mbar_init(&v_full[b], 4); mbar_init(&v_empty[b], 1); }       // 4 value producer warps
-        for (int r = 0; r < nrec; ++r) { mbar_init(&r_full[r], 1); mbar_init(&r_empty[r], 4); }
+        for (int b = 0; b < kring; ++b) { mbar_init(&k_full[b], 8); mbar_init(&k_empty[b], 1); }   // 8 producer warps
+        for (int b = 0; b < 2; ++b) { mbar_init(&v_full[b], 4); mbar_init(&v_empty[b], 1); }       // 4 per tile half
+        for (int r = 0; r < nrec; ++r) { mbar_init(&r_full[r], 1); mbar_init(&r_empty[r], 8); }
         mbar_init(s_full, 1);
         mbar_init(s_empty, 4);
         for (int b = 0; b < 2; ++b) {
@@ -218,8 +218,10 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
                 if (TWO) bulk_load(R + (size_t)kAtTok * sbytes, codes + (g * T_len + t0) * cbytes, cb, &r_full[rs]);
             }
         }
-    } else if (pidx >= 0 && pidx < 4) {
-        // ------------------------------------------------------------ key producers (thread = rows r, r + 128)
+    } else if (pidx >= 0) {
+        // ------------------------------------------------------------ producers (thread = token row)
+        const int r = pidx * 32 + lane;                           // 0..255
+        const int vh = r >> 7, vr = r & 127;                      // value slice (tile half) and row in it
         const float kq = 1.2533141373155002512f / (float)m;
         const uint32_t lane8 = (uint32_t)(lane & 7);
         int64_t slice = 0;
@@ -227,66 +229,74 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
             const int64_t k = it - it0;
             const int rs = (int)(k % nrec);
             const int64_t g = it / tiles_per_g, t0 = (it % tiles_per_g) * kAtTok;
-            uint32_t rho2[2] = {0x3C003C00u, 0x3C003C00u};
-            if (TWO) {
+            const bool tv = t0 + r < T_len;
+            const int64_t kt = g * T_len + t0 + r;
+            // the value row's codes and norm (loaded early, used after the keys)
+            uint32_t vw[vcb / 4];
+            uint32_t vf2 = 0u;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int r = pidx * 32 + lane + 128 * h;
-                    float rho = 0.0f;
-                    if (t0 + r < T_len) {
-                        const int64_t kt = g * T_len + t0 + r;
-                        const float n1 = h16_to_f32(__ldg(norms + kt));
-                        const float rn = h16_to_f32(__ldg(sk_norms + kt));
-                        if (n1 > 0.0f) rho = __fdiv_rn(__fmul_rn(__fmul_rn(kq, rn), (float)d), n1);
-                    }
-                    const uint32_t hh = (uint32_t)__half_as_ushort(__float2half_rn(rho));
-                    rho2[h] = hh | (hh << 16);
+            for (int i = 0; i < (int)(vcb / 16); ++i) {
+                const uint4 v4 = tv ? __ldg(reinterpret_cast<const uint4 *>(vcodes + kt * vcb) + i) : make_uint4(0u, 0u, 0u, 0u);
+                vw[4 * i] = v4.x; vw[4 * i + 1] = v4.y; vw[4 * i + 2] = v4.z; vw[4 * i + 3] = v4.w;
+            }
+            if (tv) {
+                const float fv = __fmul_rn(h16_to_f32(__ldg(vnorms + kt)), 1.0f / (float)kAtD);
+                const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(fv));
+                vf2 = h | (h << 16);
+            }
+            uint32_t rho2 = 0x3C003C00u;
+            if (TWO) {
+                float rho = 0.0f;
+                if (tv) {
+                    const float n1 = h16_to_f32(__ldg(norms + kt));
+                    const float rn = h16_to_f32(__ldg(sk_norms + kt));
+                    if (n1 > 0.0f) rho = __fdiv_rn(__fmul_rn(__fmul_rn(kq, rn), (float)d), n1);
                 }
+                const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(rho));
+                rho2 = h | (h << 16);
             }
             if (ok && !mbar_wait(&r_full[rs], (uint32_t)((k / nrec) & 1))) ok = false;
             const uint8_t *R = sR + (size_t)rs * rec_stride;
+            const uint8_t *Rs = R + (size_t)r * sbytes;
+            const uint8_t *Rc = R + (size_t)kAtTok * sbytes + (size_t)r * cbytes;
             for (int s = 0; s < nsl; ++s, ++slice) {
                 const int b = (int)(slice % kring);
                 const int64_t use = slice / kring;
                 if (use > 0 && ok && !mbar_wait(&k_empty[b], (uint32_t)((use - 1) & 1))) ok = false;
+                uint8_t *Br = sK + (size_t)b * kAtKSlice + (size_t)(r >> 3) * 1024 + (size_t)(r & 7) * 128;
+                if (TWO && s < dsl) {
+                    uint32_t cw[2 * PW];
+                    const uint8_t *cp = Rc + s * 8 * PW;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int r = pidx * 32 + lane + 128 * h;
-                    uint8_t *Br = sK + (size_t)b * kAtKSlice + (size_t)(r >> 3) * 1024 + (size_t)(r & 7) * 128;
-                    if (TWO && s < dsl) {
-                        uint32_t cw[2 * PW];
-                        const uint8_t *cp = R + (size_t)kAtTok * sbytes + (size_t)r * cbytes + s * 8 * PW;
+                    for (int q = 0; q < PW; ++q) {
+                        const uint2 v2 = *reinterpret_cast<const uint2 *>(cp + 8 * q);
+                        cw[2 * q] = v2.x;
+                        cw[2 * q + 1] = v2.y;
+                    }
 #pragma unroll
-                        for (int q = 0; q < PW; ++q) {
-                            const uint2 v2 = *reinterpret_cast<const uint2 *>(cp + 8 * q);
-                            cw[2 * q] = v2.x;
-                            cw[2 * q + 1] = v2.y;
-                        }
+                    for (int kk = 0; kk < 8; ++kk) {
+                        uint32_t o[4];
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            uint32_t o[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const uint32_t ca = unpack_code<64, PW>(cw, 8 * kk + 2 * e);
-                                const uint32_t cb2 = unpack_code<64, PW>(cw, 8 * kk + 2 * e + 1);
-                                if constexpr (PW <= 4) {
-                                    o[e] = klut[((ca | (cb2 << PW)) << 3) + lane8];
-                                } else {
-                                    const uint16_t *k16 = reinterpret_cast<const uint16_t *>(klut);
-                                    o[e] = (uint32_t)k16[(ca << 3) + lane8] | ((uint32_t)k16[(cb2 << 3) + lane8] << 16);
-                                }
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t ca = unpack_code<64, PW>(cw, 8 * kk + 2 * e);
+                            const uint32_t cb2 = unpack_code<64, PW>(cw, 8 * kk + 2 * e + 1);
+                            if constexpr (PW <= 4) {
+                                o[e] = klut[((ca | (cb2 << PW)) << 3) + lane8];
+                            } else {
+                                const uint16_t *k16 = reinterpret_cast<const uint16_t *>(klut);
+                                o[e] = (uint32_t)k16[(ca << 3) + lane8] | ((uint32_t)k16[(cb2 << 3) + lane8] << 16);
                             }
-                            *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                         }
-                    } else {
-                        const int sc0 = (s - dsl) * 64;
-                        const uint2 v2 = *reinterpret_cast<const uint2 *>(R + (size_t)r * sbytes + sc0 / 8);
-                        const uint32_t sb[2] = {v2.x, v2.y};
+                        *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                } else {
+                    const int sc0 = (s - dsl) * 64;
+                    const uint2 v2 = *reinterpret_cast<const uint2 *>(Rs + sc0 / 8);
+                    const uint32_t sb[2] = {v2.x, v2.y};
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t byte = (sb[kk >> 2] >> (8 * (kk & 3))) & 0xffu;
-                            *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = signs8_to_h2x4(byte, rho2[h]);
-                        }
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t byte = (sb[kk >> 2] >> (8 * (kk & 3))) & 0xffu;
+                        *reinterpret_cast<uint4 *>(Br + ((kk ^ (r & 7)) << 4)) = signs8_to_h2x4(byte, rho2);
                     }
                 }
                 fence_proxy_async_smem();
@@ -295,59 +305,34 @@ attention_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&r_empty[rs]);
-        }
-    } else if (pidx >= 4) {
-        // ------------------------------------------------------------ value producers (thread = rows r, r + 128)
-        const uint32_t lane8 = (uint32_t)(lane & 7);
-        const int vr = (pidx - 4) * 32 + lane;                   // row in each 128-token value slice
-        for (int64_t it = it0; it < it1 && ok; ++it) {
-            const int64_t k = it - it0;
-            const int64_t g = it / tiles_per_g, t0 = (it % tiles_per_g) * kAtTok;
-#pragma unroll 1
-            for (int vh = 0; vh < 2; ++vh) {
-                const int r = vh * 128 + vr;
-                const bool tv = t0 + r < T_len;
-                const int64_t kt = g * T_len + t0 + r;
-                uint32_t vw[vcb / 4];
-                uint32_t vf2 = 0u;
+            // value row: V' = fp16(c) * fp16(n / d), rows of the MN-major B operand (two 64-wide atoms of d)
+            if (k > 0 && ok && !mbar_wait(&v_empty[vh], (uint32_t)((k - 1) & 1))) ok = false;
+            uint8_t *Vr = sV + (size_t)vh * kAtVSlice + (size_t)(vr >> 3) * 1024 + (size_t)(vr & 7) * 128;
 #pragma unroll
-                for (int i = 0; i < (int)(vcb / 16); ++i) {
-                    const uint4 v4 = tv ? __ldg(reinterpret_cast<const uint4 *>(vcodes + kt * vcb) + i) : make_uint4(0u, 0u, 0u, 0u);
-                    vw[4 * i] = v4.x; vw[4 * i + 1] = v4.y; vw[4 * i + 2] = v4.z; vw[4 * i + 3] = v4.w;
-                }
-                if (tv) {
-                    const float fv = __fmul_rn(h16_to_f32(__ldg(vnorms + kt)), 1.0f / (float)kAtD);
-                    const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(fv));
-                    vf2 = h | (h << 16);
-                }
-                if (k > 0 && ok && !mbar_wait(&v_empty[vh], (uint32_t)((k - 1) & 1))) ok = false;
-                uint8_t *Vr = sV + (size_t)vh * kAtVSlice + (size_t)(vr >> 3) * 1024 + (size_t)(vr & 7) * 128;
+            for (int ch = 0; ch < 16; ++ch) {                     // 16 chunks of 8 values: d = 8 ch ... 8 ch + 7
+                uint32_t o[4];
 #pragma unroll
-                for (int ch = 0; ch < 16; ++ch) {                 // 16 chunks of 8 values: d = 8 ch ... 8 ch + 7
-                    uint32_t o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 8 * ch + 2 * e;
-                        const uint32_t ca = unpack_code<kAtD, VPW>(vw, j), cb2 = unpack_code<kAtD, VPW>(vw, j + 1);
-                        uint32_t pr;
-                        if constexpr (VPW <= 4) {
-                            pr = vlut[((ca | (cb2 << VPW)) << 3) + lane8];
-                        } else {
-                            const uint16_t *v16 = reinterpret_cast<const uint16_t *>(vlut);
-                            pr = (uint32_t)v16[(ca << 3) + lane8] | ((uint32_t)v16[(cb2 << 3) + lane8] << 16);
-                        }
-                        const __half2 hv = __hmul2(*reinterpret_cast<const __half2 *>(&pr),
-                                                   *reinterpret_cast<const __half2 *>(&vf2));
-                        o[e] = tv ? *reinterpret_cast<const uint32_t *>(&hv) : 0u;
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 8 * ch + 2 * e;
+                    const uint32_t ca = unpack_code<kAtD, VPW>(vw, j), cb2 = unpack_code<kAtD, VPW>(vw, j + 1);
+                    uint32_t pr;
+                    if constexpr (VPW <= 4) {
+                        pr = vlut[((ca | (cb2 << VPW)) << 3) + lane8];
+                    } else {
+                        const uint16_t *v16 = reinterpret_cast<const uint16_t *>(vlut);
+                        pr = (uint32_t)v16[(ca << 3) + lane8] | ((uint32_t)v16[(cb2 << 3) + lane8] << 16);
                     }
-                    const int atom = ch >> 3, c8 = ch & 7;
-                    *reinterpret_cast<uint4 *>(Vr + (size_t)atom * (kAtVSlice / 2) + ((c8 ^ (vr & 7)) << 4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
+                    const __half2 hv = __hmul2(*reinterpret_cast<const __half2 *>(&pr),
+                                               *reinterpret_cast<const __half2 *>(&vf2));
+                    o[e] = tv ? *reinterpret_cast<const uint32_t *>(&hv) : 0u;
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&v_full[vh]);
+                const int atom = ch >> 3, c8 = ch & 7;
+                *reinterpret_cast<uint4 *>(Vr + (size_t)atom * (kAtVSlice / 2) + ((c8 ^ (vr & 7)) << 4)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&v_full[vh]);
         }
     } else if (warp == 11) {
         // ------------------------------------------------------------ MMA 1: S = A_q . K

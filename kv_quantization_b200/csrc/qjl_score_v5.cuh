@@ -33,11 +33,16 @@
 //   warps 8-15 (epilogue): warp w reads TMEM lane quarter w % 4 (queries)
 //                        and columns 128 ((w - 8) / 4) ... of the tile, scales
 //                        them (per-token factors loaded one tile ahead) and
-//                        stores 16-byte runs of scores[g][q][t].
+//                        stores them: when n_q <= 64 and T % 4 == 0 through
+//                        a swizzled 16 x 32 stage and one TMA store per box
+//                        (a {T, n_q, G} tensor map, so no box crosses a
+//                        group), else as 16-byte runs of scores[g][q][t].
 // With n_q <= 64 the MMAs are M = 64: half the A operand is read per
 // instruction, and the 64 rows spread over the four lane quarters (16 each),
 // so that up to four quarters' epilogue warps share the output.
 #pragma once
+#include <cuda.h>
+
 #include "qjl_score_v4.cuh"
 
 namespace rq {
@@ -60,11 +65,15 @@ __host__ __device__ inline size_t sc5_rec_bytes(int d, int m, bool two, int pw)
 {
     return (size_t)kSc5Tok * ((size_t)m / 8 + (two ? (size_t)d * pw / 8 : 0));
 }
-__host__ __device__ inline size_t sc5_smem(int nq, int d, int m, bool two, int pw, int ring, int nrec)
+// TMA-store stage of the epilogue: per epilogue warp two 16-row x 32-float
+// boxes (128-byte swizzle), used when n_q <= 64 and T % 4 == 0.
+constexpr size_t kSc5StageBytes = (size_t)8 * 2 * 16 * 128;
+__host__ __device__ inline size_t sc5_smem(int nq, int d, int m, bool two, int pw, int ring, int nrec, bool tma)
 {
     const int kb = sc2_kb(d, m, two);
     size_t b = 1024;
     b += (sc5_a_bytes(nq, kb) + 1023) & ~(size_t)1023;            // A (queries)
+    if (tma) b += kSc5StageBytes;                                  // output stage
     b += (size_t)ring * kSc5SliceBytes;                            // B ring (also absorbs the A overrun)
     b += (size_t)nrec * ((sc5_rec_bytes(d, m, two, pw) + 127) & ~(size_t)127);   // records
     if (two) b += pw <= 4 ? ((size_t)1 << (2 * pw)) * 32 * 4 : ((size_t)1 << pw) * 32 * 2;
@@ -101,7 +110,8 @@ __global__ void __launch_bounds__(kSc5Threads, 1)
 score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN, int nq, int d, int m,
                 const uint8_t *__restrict__ signs, const uint16_t *__restrict__ sk_norms, int64_t T_len,
                 int64_t G, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ norms,
-                const __grid_constant__ QuantTables T, float *__restrict__ scores, int ring, int nrec)
+                const __grid_constant__ QuantTables T, float *__restrict__ scores, int ring, int nrec,
+                const __grid_constant__ CUtensorMap tmo, int use_tma)
 {
     const int kb = sc2_kb(d, m, TWO);
     const int nsl = kb / 64;                         // 64-column slices per tile
@@ -113,7 +123,8 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *sA = base;
-    uint8_t *sB = sA + ((sc5_a_bytes(nq, kb) + 1023) & ~(size_t)1023);
+    uint8_t *sStage = sA + ((sc5_a_bytes(nq, kb) + 1023) & ~(size_t)1023);
+    uint8_t *sB = sStage + (use_tma ? kSc5StageBytes : 0);
     uint8_t *sR = sB + (size_t)ring * kSc5SliceBytes;
     uint32_t *clut = reinterpret_cast<uint32_t *>(sR + (size_t)nrec * rec_stride);
     const size_t clut_bytes = TWO ? (PW <= 4 ? ((size_t)1 << (2 * PW)) * 32 * 4 : ((size_t)1 << PW) * 32 * 2) : 0;
@@ -328,6 +339,8 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
         const float inv_d = 1.0f / (float)d;
         const uint16_t *nsrc = TWO ? norms : sk_norms;
         float *fac = sF + (warp - 8) * 128;                 // this warp's per-token factors
+        uint8_t *stage = sStage + (size_t)(warp - 8) * 2 * 16 * 128;   // two 2 KB boxes (use_tma)
+        int nstored = 0;                                     // boxes this warp has stored
         int64_t qn_g = -1;
         float qn = 0.0f;
         // lane l holds the factors of tokens 4 l ... 4 l + 3 of the warp's 128 columns; the next
@@ -368,7 +381,31 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
                               rr);
                     tmem_ld_wait();
                     const int64_t tc0 = tb + c * 32;
-                    if (lane_ok) {
+                    if (use_tma) {
+                        // rows 16 quarter ... of the box: this lane's 32 scores, 128-byte swizzled
+                        uint8_t *box = stage + (size_t)(nstored & 1) * 2048;
+                        if (lane == 0 && nstored >= 2) bulk_wait_read<1>();    // the box's previous store has read it
+                        __syncwarp();
+                        if (lane < 16) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4) {
+                                const float4 fv = *reinterpret_cast<const float4 *>(fac + c * 32 + i);
+                                float4 v;
+                                v.x = __fmul_rn(__fmul_rn(fv.x, __uint_as_float(rr[i])), qn);
+                                v.y = __fmul_rn(__fmul_rn(fv.y, __uint_as_float(rr[i + 1])), qn);
+                                v.z = __fmul_rn(__fmul_rn(fv.z, __uint_as_float(rr[i + 2])), qn);
+                                v.w = __fmul_rn(__fmul_rn(fv.w, __uint_as_float(rr[i + 3])), qn);
+                                *reinterpret_cast<float4 *>(box + sw128_offset((uint32_t)lane, (uint32_t)(i >> 2))) = v;
+                            }
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {                               // boxes with no column inside T are skipped
+                            if (tc0 < T_len) tma_store_3d(&tmo, (int)tc0, quarter * 16, (int)g, box);
+                            bulk_commit();
+                        }
+                        ++nstored;
+                    } else if (lane_ok) {
                         float *dst = dst0 + tc0;
                         const bool full = tc0 + 32 <= T_len && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
 #pragma unroll
@@ -396,6 +433,7 @@ score_v5_kernel(const uint16_t *__restrict__ wsB, const float *__restrict__ wsN,
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[a]);
         }
+        if (use_tma && lane == 0) bulk_wait<0>();              // every store has completed before exit
     }
     tc_fence_before();
     __syncthreads();

@@ -357,6 +357,19 @@ bool rq::make_proj_tmap(CUtensorMap *map, const void *ptr, int m, int d, int box
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool rq::make_scores_tmap(CUtensorMap *map, const void *ptr, int64_t T, int nq, int64_t G)
+{
+    auto enc = tmap_encoder();
+    if (!enc || T <= 0 || T % 4 || T >= ((int64_t)1 << 31) || nq <= 0 || G <= 0) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)T, (cuuint64_t)nq, (cuuint64_t)G};
+    const cuuint64_t strides[2] = {(cuuint64_t)T * 4, (cuuint64_t)T * 4 * (cuuint64_t)nq};
+    const cuuint32_t box[3] = {32, 16, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 extern "C" {
 
 const char *rq_status_string(int status)
@@ -652,6 +665,7 @@ rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void 
     a.codes = static_cast<const uint8_t *>(codes); a.norms = norms; a.pw = pw; a.tables = &T;
     a.scores = scores; a.workspace = static_cast<float *>(workspace); a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
+    a.has_tmap_scores = rq::make_scores_tmap(&a.tmap_scores, scores, T_len, n_q, G);
     return cuda_status(rq::launch_score(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

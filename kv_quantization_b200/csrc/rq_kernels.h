@@ -74,6 +74,8 @@ struct ScoreArgs {
     int pw;
     const QuantTables *tables;
     float *scores;             // [G][nq][T]
+    CUtensorMap tmap_scores;   // make_scores_tmap, when has_tmap_scores
+    bool has_tmap_scores;
     float *workspace;          // [G][nq][d + m] fp32
     int num_sms;
 };
@@ -119,6 +121,9 @@ bool make_rows64_tmap(CUtensorMap *map, const void *ptr, int64_t rows);
 bool make_vectors_tmap(CUtensorMap *map, const void *ptr, int64_t n, int d, int box_rows = 128);
 // Encode S[m][d] (16-bit) with {64 columns, box_rows rows} boxes (B operand layout).
 bool make_proj_tmap(CUtensorMap *map, const void *ptr, int m, int d, int box_rows);
+// fp32 scores [G][nq][T] as a {T, nq, G} map with 32 x 16 x 1 boxes (128-byte
+// swizzle), for TMA stores that never cross a group; needs T % 4 == 0.
+bool make_scores_tmap(CUtensorMap *map, const void *ptr, int64_t T, int nq, int64_t G);
 size_t dequantize_smem_bytes(int d);
 // One CTA that waits, at most `polls` times, on an mbarrier nothing arrives
 // on, then unwinds as the tensor-core kernels do (rq_probe_bounded_wait).

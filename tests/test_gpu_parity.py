@@ -443,3 +443,41 @@ def test_score_two_stage_shapes(d, bits, m, nq, layout):
                    codes=codes.cpu().numpy(), norms=n16, bits=bits, layout=layout,
                    signs_diag=O.sign_diagonal(9, d), c32=cent)
     check_scores(scores.cpu().numpy(), want, score_tol(q16, G, nq, d, n16), f"two-stage d={d} b={bits} nq={nq}")
+
+
+@pytest.mark.parametrize("two,nq,T", [(False, 24, 1000), (True, 40, 2052), (False, 64, 516)])
+def test_score_tma_store_shapes(two, nq, T):
+    """T % 4 == 0 takes the score kernel's TMA-store epilogue: ragged last
+    boxes (T not a multiple of 32) and query counts that end inside a
+    16-row box are clipped by the tensor map, never written past a group."""
+    G, d, bits = 3, 128, 2
+    m = 128 if two else 256
+    q = synth.normal((G, nq, d), seed=31, device=DEV)
+    scores = torch.full((G, nq, T), float("nan"), dtype=torch.float32, device=DEV)
+    ws = torch.empty(L.qjl_score_workspace_bytes(G, nq, d, m) // 4, dtype=torch.float32, device=DEV)
+    q16 = u16(q)
+    if two:
+        k, cent, S, codes, norms, qs, qn = make_two_stage(G, T, d, bits, m, L.RQ_CODES_PACKED, 32, 33, 34)
+        L.qjl_score(q, G, nq, d, m, S, qs, qn, T, scores, ws, codes=codes, norms=norms, bits=bits,
+                    layout=L.RQ_CODES_PACKED, use_signs=1, sign_seed=33, centroids=cent)
+        n16 = norms.cpu().numpy().view(np.uint16)
+        want = O.score(q16, G, nq, d, m, u16(S), O.BF16, qs.cpu().numpy(), qn.cpu().numpy().view(np.uint16), T,
+                       codes=codes.cpu().numpy(), norms=n16, bits=bits, layout=O.PACKED,
+                       signs_diag=O.sign_diagonal(33, d), c32=cent)
+        tol = score_tol(q16, G, nq, d, n16)
+    else:
+        k = synth.kv_with_channels(1, G, T, d, seed=35, device=DEV).reshape(-1)
+        S = torch.empty(m, d, dtype=torch.bfloat16, device=DEV)
+        L.qjl_make_projection(36, m, d, S)
+        signs = torch.empty(G * T * m // 8, dtype=torch.uint8, device=DEV)
+        kn = torch.empty(G * T, dtype=torch.int16, device=DEV)
+        L.qjl_sketch(k, d, m, S, signs, kn)
+        L.qjl_score(q, G, nq, d, m, S, signs, kn, T, scores, ws)
+        kn16 = kn.cpu().numpy().view(np.uint16)
+        want = O.score(q16, G, nq, d, m, u16(S), O.BF16, signs.cpu().numpy(), kn16, T)
+        tol = score_tol(q16, G, nq, d, kn16)
+    assert L.rq_last_launch() == "score_v2_prologue,score_v5_kernel"
+    torch.cuda.synchronize()
+    got = scores.cpu().numpy()
+    assert not np.isnan(got).any()
+    check_scores(got, want, tol, f"tma store two={two} nq={nq} T={T}")
