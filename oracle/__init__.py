@@ -72,6 +72,7 @@ def lib():
                 "orc_attention": (i32, [u16, i64, i32, i32, i32, u16, i32, u8, u16, i64,
                                         u8, u16, i32, i32, i8, f32,
                                         u8, u16, i32, i32, i8, f32, C.c_double, f64]),
+                "orc_sub_blocks": (i32, [i32, C.POINTER(C.c_int), C.POINTER(C.c_int)]),
                 "orc_unpack_codes": (None, [u8, i64, i32, i32, i32, u8]),
                 "orc_pack_codes": (None, [u8, i64, i32, i32, i32, u8]),
                 "orc_hadamard_matrix": (None, [i32, f64]),
@@ -279,6 +280,15 @@ def attention(q16, G, nq, d, m, S16, sdtype, signs, sk_norms, T, vcodes, vnorms,
     if rc != 0:
         raise ValueError("orc_attention: empty key range")
     return out.reshape(G, nq, d)
+
+
+def sub_blocks(d):
+    """orc_sub_blocks -> [(offset, size), ...]: the power-of-two sub-blocks of a
+    block of d values, largest first."""
+    off = (C.c_int * 31)()
+    sz = (C.c_int * 31)()
+    n = lib().orc_sub_blocks(d, off, sz)
+    return [(off[i], sz[i]) for i in range(n)]
 
 
 def unpack_codes(codes, nblocks, d, bits, layout):

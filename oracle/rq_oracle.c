@@ -262,11 +262,30 @@ static float pairwise_sum(const float *v, int n)
     return a + b;
 }
 
-/* fp32 L2 norm: squares rounded to fp32, pairwise sum, correctly rounded sqrt. */
+/* Sub-blocks of a block of d values: the binary decomposition of d, largest
+ * power of two first (GLQ README, "Bit widths": a non-power-of-two size such as
+ * 2688 is decomposed as 2048 + 512 + 128 and transformed block-diagonally;
+ * turbopress "Package layout": block-diagonal Walsh-Hadamard times Rademacher
+ * signs, an orthogonal transform).  A power of two is one sub-block.
+ * Returns the count; off[] and sz[] receive offsets and sizes (at most 31). */
+int orc_sub_blocks(int d, int *off, int *sz)
+{
+    int n = 0, o = 0;
+    for (int b = 1 << 30; b >= 1; b >>= 1)
+        if (d - o >= b) { off[n] = o; sz[n] = b; o += b; ++n; }
+    return n;
+}
+
+/* fp32 L2 norm: squares rounded to fp32, pairwise sum within each sub-block,
+ * the sub-block sums added in order, correctly rounded sqrt. */
 static float norm_f32(const float *v, int d, float *tmp)
 {
+    int off[31], sz[31];
+    int nb = orc_sub_blocks(d, off, sz);
     for (int j = 0; j < d; ++j) tmp[j] = v[j] * v[j];
-    return sqrtf(pairwise_sum(tmp, d));
+    float acc = pairwise_sum(tmp + off[0], sz[0]);
+    for (int i = 1; i < nb; ++i) acc = acc + pairwise_sum(tmp + off[i], sz[i]);
+    return sqrtf(acc);
 }
 
 /* Unnormalised Walsh-Hadamard transform, Sylvester (natural) order, in place:
@@ -292,6 +311,24 @@ static void fwht_f64(double *v, int d)
                 v[j + h] = a - b;
             }
 }
+
+/* Block-diagonal transform of a block of d values: fwht of every sub-block. */
+static void rotate_f32(float *v, int d)
+{
+    int off[31], sz[31];
+    int nb = orc_sub_blocks(d, off, sz);
+    for (int i = 0; i < nb; ++i) fwht_f32(v + off[i], sz[i]);
+}
+
+/* Per-sub-block scales of the block-diagonal rotation.  With R the orthogonal
+ * blockdiag(H_b / sqrt(b)) D, the quantized coordinates are
+ * y = sqrt(d) R x / ||x|| and the reconstruction x^ = ||x|| R^T c / sqrt(d):
+ *   y_j  = w_j * fl32(g_b * inv),   g_b = fl32(sqrt(d / b)),
+ *   x^_j = s_j * (w'_j * fl32(n16 * h_b)),   h_b = fl32(1 / sqrt(d b)),
+ * w = H_b D x and w' = H_b c in fp32 stages.  For a power-of-two d (one
+ * sub-block) g = 1 and h = 1/d exactly: the plain path. */
+static float sub_g(int d, int b) { return (float)sqrt((double)d / (double)b); }
+static float sub_h(int d, int b) { return (float)(1.0 / sqrt((double)d * (double)b)); }
 
 /* ------------------------------------------------------------------ */
 /* Code storage ([PQ] int8 index; [TQ] packed, low bits first).         */
@@ -364,10 +401,14 @@ int orc_quantize(const uint16_t *x, int dtype, int64_t nblocks, int d, int bits,
         norms[b] = norm_to_f16(n32);
         if (n32_out) n32_out[b] = n32;
         if (s) for (int j = 0; j < d; ++j) if (s[j] < 0) v[j] = -v[j];
-        fwht_f32(v, d);
+        rotate_f32(v, d);
         float inv = n32 > 0.0f ? 1.0f / n32 : 0.0f;
+        int off[31], sz[31];
+        int nsb = orc_sub_blocks(d, off, sz), sb = 0;
+        float f = sub_g(d, sz[0]) * inv;
         for (int j = 0; j < d; ++j) {
-            float y = v[j] * inv;
+            if (sb + 1 < nsb && j == off[sb + 1]) { ++sb; f = sub_g(d, sz[sb]) * inv; }
+            float y = v[j] * f;
             unsigned code = 0;
             for (int k = 0; k + 1 < K; ++k) code += (t[k] < y) ? 1u : 0u;
             put_code(codes + b * cb, j, bits, layout, code);
@@ -378,11 +419,14 @@ int orc_quantize(const uint16_t *x, int dtype, int64_t nblocks, int d, int bits,
     return 0;
 }
 
-/* fp64 rotated coordinates y = H D x / ||x|| (the exact-arithmetic value the
- * fp32 canonical y approximates); used to count near-boundary coordinates. */
+/* fp64 rotated coordinates y = sqrt(d) R x / ||x|| (the exact-arithmetic value
+ * the fp32 canonical y approximates; R as above, H D x / ||x|| for a power of
+ * two); used to count near-boundary coordinates. */
 int orc_rotate_f64(const uint16_t *x, int dtype, int64_t nblocks, int d, const int8_t *s, double *y_out)
 {
     double *v = (double *)malloc(sizeof(double) * (size_t)d);
+    int off[31], sz[31];
+    int nsb = orc_sub_blocks(d, off, sz);
     for (int64_t b = 0; b < nblocks; ++b) {
         double ss = 0.0;
         for (int j = 0; j < d; ++j) {
@@ -390,9 +434,12 @@ int orc_rotate_f64(const uint16_t *x, int dtype, int64_t nblocks, int d, const i
             ss += v[j] * v[j];
             if (s && s[j] < 0) v[j] = -v[j];
         }
-        fwht_f64(v, d);
         double n = sqrt(ss);
-        for (int j = 0; j < d; ++j) y_out[b * d + j] = n > 0.0 ? v[j] / n : 0.0;
+        for (int i = 0; i < nsb; ++i) {
+            fwht_f64(v + off[i], sz[i]);
+            double g = sqrt((double)d / (double)sz[i]);
+            for (int j = off[i]; j < off[i] + sz[i]; ++j) y_out[b * d + j] = n > 0.0 ? v[j] * g / n : 0.0;
+        }
     }
     free(v);
     return 0;
@@ -403,11 +450,15 @@ static void dequant_block_f32(const uint8_t *field, uint16_t norm16, int d, int 
                               const int8_t *s, const float *c, float *w)
 {
     for (int j = 0; j < d; ++j) w[j] = c[get_code(field, j, bits, layout)];
-    fwht_f32(w, d);
-    float scale = orc_f16_to_f32(norm16) / (float)d;      /* exact: d is a power of two */
-    for (int j = 0; j < d; ++j) {
-        float xh = w[j] * scale;
-        w[j] = (s && s[j] < 0) ? -xh : xh;
+    rotate_f32(w, d);
+    int off[31], sz[31];
+    int nsb = orc_sub_blocks(d, off, sz);
+    for (int i = 0; i < nsb; ++i) {
+        float scale = orc_f16_to_f32(norm16) * sub_h(d, sz[i]);   /* n16 / d exactly for a power of two */
+        for (int j = off[i]; j < off[i] + sz[i]; ++j) {
+            float xh = w[j] * scale;
+            w[j] = (s && s[j] < 0) ? -xh : xh;
+        }
     }
 }
 
@@ -434,13 +485,17 @@ int orc_dequantize_f64(const uint8_t *codes, const uint16_t *norms, int64_t nblo
 {
     double *w = (double *)malloc(sizeof(double) * (size_t)d);
     int64_t cb = block_code_bytes(d, bits, layout);
+    int off[31], sz[31];
+    int nsb = orc_sub_blocks(d, off, sz);
     for (int64_t b = 0; b < nblocks; ++b) {
         for (int j = 0; j < d; ++j) w[j] = c[get_code(codes + b * cb, j, bits, layout)];
-        fwht_f64(w, d);
         double n = orc_f16_to_f32(norms[b]);
-        for (int j = 0; j < d; ++j) {
-            double xh = w[j] * n / d;
-            out[b * d + j] = (s && s[j] < 0) ? -xh : xh;
+        for (int i = 0; i < nsb; ++i) {
+            fwht_f64(w + off[i], sz[i]);
+            for (int j = off[i]; j < off[i] + sz[i]; ++j) {
+                double xh = w[j] * n / sqrt((double)d * (double)sz[i]);
+                out[b * d + j] = (s && s[j] < 0) ? -xh : xh;
+            }
         }
     }
     free(w);
@@ -519,6 +574,7 @@ int orc_score(const uint16_t *q, int64_t G, int nq, int d, int m, const uint16_t
               const uint8_t *codes, const uint16_t *norms, int bits, int layout,
               const int8_t *s, const float *c, double *scores)
 {
+    if (codes && (d & (d - 1))) return -1;     /* two-stage scores: power-of-two blocks only */
     double *qv = (double *)malloc(sizeof(double) * (size_t)d);
     double *qt = (double *)malloc(sizeof(double) * (size_t)d);
     double *sq = (double *)malloc(sizeof(double) * (size_t)m);

@@ -494,3 +494,68 @@ def test_attention_token_permutation_invariant_and_hard_limit():
     vh = O.dequantize_f64(c["vcodes"], c["vnorms"], d, vbits, O.PACKED, c["vs"], c["vc"]).reshape(T, d)
     assert np.all(np.isfinite(hard))
     assert np.allclose(hard, vh[top[:, -1]], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ non-power-of-two blocks
+
+def test_sub_blocks_follow_the_printed_decomposition():
+    for row in read_golden("block_diagonal_sizes.txt"):
+        d, want = int(row[0]), [int(v) for v in row[1:]]
+        assert [b for _, b in O.sub_blocks(d)] == want
+    for d in (96, 160, 192, 224, 320, 448, 480, 128, 512):
+        sb = O.sub_blocks(d)
+        sizes = [b for _, b in sb]
+        assert sum(sizes) == d and sizes == sorted(sizes, reverse=True)
+        assert all(b & (b - 1) == 0 for b in sizes) and len(set(sizes)) == len(sizes)
+        assert [o for o, _ in sb] == [sum(sizes[:i]) for i in range(len(sizes))]
+
+
+def _rotation_matrix(d, signs):
+    """sqrt(d) blockdiag(H_b / sqrt(b)) D from scipy's Sylvester Hadamard."""
+    blocks = [scipy.linalg.hadamard(b) / math.sqrt(b) for _, b in O.sub_blocks(d)]
+    return math.sqrt(d) * scipy.linalg.block_diag(*blocks) @ np.diag(signs.astype(np.float64))
+
+
+@pytest.mark.parametrize("d", [96, 192, 320, 448])
+def test_block_diagonal_rotation_matches_scipy(d):
+    """y = sqrt(d) R x / ||x|| with R = blockdiag(H_b / sqrt(b)) D orthogonal:
+    the fp64 rotation against scipy's Hadamard, ||y|| = sqrt(d), and the fp32
+    canonical coordinates within a few ulps of it."""
+    rng = np.random.default_rng(d)
+    n = 7
+    x = rand_u16(rng, n * d, 1.0, O.BF16)
+    s = O.sign_diagonal(11, d)
+    R = _rotation_matrix(d, s)
+    assert np.allclose(R @ R.T, d * np.eye(d), atol=1e-9)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(n, d)
+    want = (xf @ R.T) / np.linalg.norm(xf, axis=1, keepdims=True)
+    y64 = O.rotate_f64(x, O.BF16, d, s).reshape(n, d)
+    assert np.allclose(y64, want, rtol=1e-12, atol=1e-12)
+    assert np.allclose(np.linalg.norm(y64, axis=1), math.sqrt(d), rtol=1e-12)
+    _, _, y32, _ = O.quantize(x, O.BF16, d, 4, O.PACKED, s, O.f32_table(4), want_y=True)
+    assert np.abs(y32.reshape(n, d) - y64).max() <= 1e-5 * np.abs(y64).max()
+
+
+@pytest.mark.parametrize("d,bits", [(96, 4), (160, 3), (448, 2)])
+def test_block_diagonal_codes_are_nearest_and_reconstruct(d, bits):
+    """Codes are the nearest centroid of the fp32 coordinates (brute force), and
+    the fp64 reconstruction is ||x||16 R^T c / sqrt(d) (scipy); the fp32 one
+    stays within 1e-6 of it relative to the block norm."""
+    rng = np.random.default_rng(d + bits)
+    n = 9
+    x = rand_u16(rng, n * d, 1.0, O.BF16)
+    s = O.sign_diagonal(12, d)
+    c = O.f32_table(bits)
+    codes, norms, y32, _ = O.quantize(x, O.BF16, d, bits, O.PACKED, s, c, want_y=True)
+    idx = O.unpack_codes(codes, n, d, bits, O.PACKED).reshape(n, d).astype(np.int64)
+    y = y32.reshape(n, d).astype(np.float64)
+    dist = np.abs(y[..., None] - c.astype(np.float64)[None, None, :])
+    best = dist.min(-1, keepdims=True)
+    assert np.all(dist[np.arange(n)[:, None], np.arange(d)[None, :], idx] <= best[..., 0] + 1e-12)
+    R = _rotation_matrix(d, s)
+    n16 = np.array([O.f16_to_f32(int(h)) for h in norms], np.float64)
+    want = (c.astype(np.float64)[idx] @ R) * (n16[:, None] / d)
+    xh64 = O.dequantize_f64(codes, norms, d, bits, O.PACKED, s, c).reshape(n, d)
+    assert np.allclose(xh64, want, rtol=1e-12, atol=1e-12)
+    _, xh32 = O.dequantize(codes, norms, d, bits, O.PACKED, s, c, O.BF16, want_f32=True)
+    assert np.abs(xh32.reshape(n, d) - xh64).max() <= 1e-6 * n16.max()
