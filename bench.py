@@ -59,7 +59,7 @@ def parse(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile", default=None,
                    help="run one case's kernels once (profiling driver): c3_layer, weight4096_fused, kv_sketch, "
-                        "kv_score, kv_attention, kv_v, tq256, tq512; print nothing else")
+                        "kv_score, kv_attention, kv_v, kv_v96, tq256, tq512; print nothing else")
     p.add_argument("--rank-selftest", action="store_true", help=argparse.SUPPRESS)
     return p.parse_args(argv)
 
@@ -485,6 +485,26 @@ def secondary_lines(dev, reps=10, only=None):
                     "roofline": roofline_hbm(alg_quant(n) + alg_dequant(n), tq + tdq)})
         del v, codes, norms, o
 
+    if want("kv_v96"):
+        # the same V line at head dim 96: blocks of a non-power-of-two size (block-diagonal 64 + 32 transform)
+        dv = 96
+        v = synth.kv_with_channels(4, 8, 32768, dv, seed=13, device=dev).reshape(-1)
+        n = v.numel()
+        cent = rq.rq_lloyd_max(4)
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        norms = torch.empty(n // dv, dtype=torch.int16, device=dev)
+        o = torch.empty_like(v)
+        q = lambda: rq.rq_quantize(v, dv, 4, rq.RQ_CODES_PACKED, 1, 14, cent, codes, norms)
+        dq = lambda: rq.rq_dequantize(codes, norms, n, dv, 4, rq.RQ_CODES_PACKED, 1, 14, cent, o)
+        q(); dq()
+        tq, tdq = median_ms(q, reps), median_ms(dq, reps)
+        out.append({"workload": "KV cache V 4x8x32768x96 bf16 N(0,1) (4 channels/head x10), head dim 96: block-diagonal "
+                                "64 + 32 RHT (signs seed 14) + 4-bit Lloyd-Max quantize then dequantize",
+                    "quantize_ms": round(tq, 4), "dequantize_ms": round(tdq, 4),
+                    "input_gbs": round(n * 2 / ((tq + tdq) * 1e-3) / 1e9, 1),
+                    "roofline": roofline_hbm(alg_quant(n, d=dv) + alg_dequant(n, d=dv), tq + tdq)})
+        del v, codes, norms, o
+
     if want("kv_k"):
         G, T, d, m, nq = 32, 32768, 128, 256, 32
         k = synth.kv_with_channels(4, 8, T, d, seed=3, device=dev).reshape(-1)
@@ -738,7 +758,7 @@ def profile_case(case):
         rq.rq_dequantize(codes, norms, LAYER_N, D, BITS, rq.RQ_CODES_PACKED, 1, 1000, cent, out)
     else:
         key = {"weight4096_fused": "weight4096", "kv_sketch": "kv_k", "kv_score": "kv_k", "kv_attention": "kv_k",
-               "kv_v": "kv_v", "tq256": "tq256", "tq512": "tq512"}[case]
+               "kv_v": "kv_v", "kv_v96": "kv_v96", "tq256": "tq256", "tq512": "tq512"}[case]
         secondary_lines(dev, reps=1, only=key)
     torch.cuda.synchronize()
     assert rq.rq_device_error(True) == 0

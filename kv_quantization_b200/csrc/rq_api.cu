@@ -236,7 +236,7 @@ rq_status make_tables(const float *centroids, int bits, int d, int use_signs, ui
     if (!build_lut(T.bound, K - 1, T)) T.lut_cells = 0;
     if (!build_sat_lut(T.bound, K - 1, T)) T.sat_cells = 0;
     if (use_signs) {
-        for (int w = 0; w < d / 64; ++w) {
+        for (int w = 0; w < (d + 63) / 64; ++w) {          // one SplitMix64 output per 64 coordinates
             const uint64_t r = splitmix64(sign_seed, (uint64_t)w);
             T.sign_words[2 * w] = (uint32_t)(r & 0xffffffffu);
             T.sign_words[2 * w + 1] = (uint32_t)(r >> 32);
@@ -388,7 +388,7 @@ const char *rq_status_string(int status)
 
 int64_t rq_code_bytes(int64_t n, int d, int bits, rq_layout layout)
 {
-    if (!pow2_d(d) || bits < 1 || bits > 8 || n < 0 || n % d) return -1;
+    if ((!pow2_d(d) && !rq::bd_size(d)) || bits < 1 || bits > 8 || n < 0 || n % d) return -1;
     if (layout == RQ_CODES_INT8) return n;
     if (layout != RQ_CODES_PACKED) return -1;
     return (n / d) * ((int64_t)d * bits / 8);
@@ -423,7 +423,7 @@ rq_status rq_lloyd_max(int bits, float *centroids_out)
 
 static rq_status check_common(int64_t n, int d, int bits, rq_layout layout)
 {
-    if (!pow2_d(d)) return (d > 0 && (d & (d - 1)) == 0) ? RQ_EUNSUPPORTED : RQ_EINVAL;
+    if (!pow2_d(d) && !rq::bd_size(d)) return d > 0 && (d & (d - 1)) == 0 ? RQ_EUNSUPPORTED : RQ_EINVAL;
     if (bits < 1 || bits > 8) return RQ_EINVAL;
     if (layout != RQ_CODES_PACKED && layout != RQ_CODES_INT8) return RQ_EINVAL;
     if (n < 0 || n % d) return RQ_EINVAL;
@@ -442,6 +442,7 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
     if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
     const bool qjl = qjl_signs != nullptr || qjl_norms != nullptr || proj != nullptr;
     if (qjl && (!qjl_signs || !qjl_norms || !proj || m < 8 || m > 512 || m % 8)) return RQ_EINVAL;
+    if (qjl && !pow2_d(d)) return RQ_EUNSUPPORTED;          // the residual sketch takes power-of-two blocks
     if (n == 0) return RQ_OK;
     if (!x || !codes || !norms) return RQ_EINVAL;
     if (!aligned16(x) || !aligned16(codes) || !aligned16(norms)) return RQ_EALIGN;
@@ -455,6 +456,7 @@ static rq_status quantize_impl(const void *x, rq_dtype dtype, int64_t n, int d, 
     a.m = qjl ? m : 0; a.proj = proj; a.qsigns = qjl_signs; a.qnorms = qjl_norms;
     a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
+    if (!pow2_d(d)) return cuda_status(rq::launch_quantize_bd(a, stream));
     if (!rq::make_rows64_tmap(&a.tmap_x, x, n / 64)) return RQ_ECUDA;
     a.has_tmap_v = qjl && rq::make_vectors_tmap(&a.tmap_v, x, n / d, d);
     a.has_tmap_v32 = !qjl && d == 128 && rq::make_vectors_tmap(&a.tmap_v32, x, n / d, d, 32);
@@ -502,6 +504,7 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
     a.bf16 = out_dtype == RQ_BF16; a.tables = &T; a.out = out;
     a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
+    if (!pow2_d(d)) return cuda_status(rq::launch_dequantize_bd(a, reinterpret_cast<cudaStream_t>(stream)));
     if (!rq::make_rows64_tmap(&a.tmap_out, out, n / 64)) return RQ_ECUDA;
     a.has_tmap_out32 = d == 128 && rq::make_vectors_tmap(&a.tmap_out32, out, n / d, d, 32);
     return cuda_status(rq::launch_dequantize(a, reinterpret_cast<cudaStream_t>(stream)));

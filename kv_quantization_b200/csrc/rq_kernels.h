@@ -87,6 +87,10 @@ void begin_call();
 void note_launch(const char *kernel);
 
 cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st);
+// Blocks of a size d that is not a power of two (rq_bd.cuh): 64 < d < 512, d % 32 == 0.
+bool bd_size(int d);
+cudaError_t launch_quantize_bd(const QuantArgs &a, cudaStream_t st);
+cudaError_t launch_dequantize_bd(const DequantArgs &a, cudaStream_t st);
 cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t st);
 cudaError_t launch_projection(uint64_t seed, int m, int d, bool bf16, void *proj, cudaStream_t st);
 cudaError_t launch_sketch(const SketchArgs &a, cudaStream_t st);

@@ -52,7 +52,9 @@ def test_code_bytes():
     assert L.rq_code_bytes(4096 * 4096, 128, 3, L.RQ_CODES_PACKED) == 4096 * 4096 * 3 // 8
     assert L.rq_code_bytes(4096 * 4096, 128, 5, L.RQ_CODES_PACKED) == 4096 * 4096 * 5 // 8
     assert L.rq_code_bytes(100, 128, 4, L.RQ_CODES_PACKED) == -1
-    assert L.rq_code_bytes(128, 96, 4, L.RQ_CODES_PACKED) == -1
+    assert L.rq_code_bytes(128, 96, 4, L.RQ_CODES_PACKED) == -1          # n not a multiple of d
+    assert L.rq_code_bytes(96 * 5, 96, 4, L.RQ_CODES_PACKED) == 96 * 5 // 2  # block-diagonal size
+    assert L.rq_code_bytes(100 * 4, 100, 4, L.RQ_CODES_PACKED) == -1     # not a multiple of 32
 
 
 def test_k_side_ratio_from_library_layout():
@@ -90,7 +92,7 @@ def _q(x, d=128, bits=4, layout=L.RQ_CODES_PACKED, cent=None, codes=None, norms=
 
 
 @pytest.mark.parametrize("case, status", [
-    (dict(d=96), -1), (dict(d=1024), -4), (dict(bits=9), -1), (dict(bits=0), -1), (dict(n=1000), -1),
+    (dict(d=100), -1), (dict(d=1024), -4), (dict(bits=9), -1), (dict(bits=0), -1), (dict(n=1000), -1),
     (dict(layout=5), -1), (dict(cent=np.array([0.0, 0.0] + [1.0] * 14, np.float32)), -1),
     (dict(cent=np.array([np.nan] * 16, np.float32)), -1),
 ])
@@ -150,7 +152,7 @@ def test_probe_and_trace_validate_before_any_launch():
     for polls in (0, (1 << 20) + 1):
         assert L.lib().rq_probe_bounded_wait(polls, None) == -1
         assert L.rq_last_launch() == ""
-    assert L.lib().rq_quantize(None, 1, 128, 96, 4, 0, 0, 0, None, None, None, None) == -1
+    assert L.lib().rq_quantize(None, 1, 128, 100, 4, 0, 0, 0, None, None, None, None) == -1
     assert L.rq_last_launch() == ""
 
 
@@ -176,3 +178,16 @@ def test_attention_validates_before_any_launch():
         with pytest.raises(L.RQError) as e:
             call(ws_numel=4)
         assert e.value.status == -5                           # stops at the device query
+
+
+def test_block_diagonal_sizes_take_no_residual_sketch():
+    """Blocks of a non-power-of-two size quantize and dequantize, but the fused
+    residual sketch takes power-of-two blocks only: RQ_EUNSUPPORTED before any
+    launch."""
+    c = O.f32_table(3)
+    with pytest.raises(L.RQError) as e:
+        L.rq_quantize_qjl(FakeTensor(0x40000), 96, 3, L.RQ_CODES_PACKED, 1, 5, c, 128, FakeTensor(0x50000),
+                          FakeTensor(0x60000), FakeTensor(0x70000), FakeTensor(0x80000), FakeTensor(0x90000),
+                          stream=0, n=96 * 64)
+    assert e.value.status == -4
+    assert L.rq_last_launch() == ""
