@@ -59,7 +59,7 @@ def parse(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile", default=None,
                    help="run one case's kernels once (profiling driver): c3_layer, weight4096_fused, kv_sketch, "
-                        "kv_score, kv_attention, kv_v, kv_v96, tq256, tq512; print nothing else")
+                        "kv_score, kv_attention, kv_v, kv_v96, kv_dense, tq256, tq512; print nothing else")
     p.add_argument("--rank-selftest", action="store_true", help=argparse.SUPPRESS)
     return p.parse_args(argv)
 
@@ -509,6 +509,32 @@ def secondary_lines(dev, reps=10, only=None):
                     "roofline": roofline_hbm(alg_quant(n, d=dv) + alg_dequant(n, d=dv), tq + tdq)})
         del v, codes, norms, o
 
+    if want("kv_dense"):
+        # the V line with a dense random orthogonal rotation (128 x 128 tensor-core GEMM per tile of
+        # 128 blocks) and the 4-bit Lloyd-Max codebook of the coordinate law of a uniform unit vector
+        v = synth.kv_with_channels(4, 8, 32768, D, seed=13, device=dev).reshape(-1)
+        n = v.numel()
+        cent = rq.rq_beta_lloyd_max(D, 4)
+        pi = torch.from_numpy(rq.rq_make_rotation(D, 17)).to(dev).to(torch.bfloat16)
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        norms = torch.empty(n // D, dtype=torch.int16, device=dev)
+        o = torch.empty_like(v)
+        q = lambda: rq.rq_quantize_dense(v, D, pi, 4, rq.RQ_CODES_PACKED, cent, codes, norms)
+        dq = lambda: rq.rq_dequantize_dense(codes, norms, n, D, pi, 4, rq.RQ_CODES_PACKED, cent, o)
+        q(); dq()
+        tq, tdq = median_ms(q, reps, batch=4), median_ms(dq, reps, batch=4)
+        flops = 2.0 * n * D                                  # one d x d rotation per block, each way
+        _, bf16_peak, _ = peaks()
+        out.append({"workload": "KV cache V 4x8x32768x128 bf16 N(0,1) (4 channels/head x10): dense random orthogonal "
+                                "rotation (QR of a Gaussian, seed 17) + 4-bit Beta-law Lloyd-Max quantize then "
+                                "dequantize",
+                    "quantize_ms": round(tq, 4), "dequantize_ms": round(tdq, 4),
+                    "input_gbs": round(n * 2 / ((tq + tdq) * 1e-3) / 1e9, 1),
+                    "tensor_tflops": round(2 * flops / ((tq + tdq) * 1e-3) / 1e12, 1),
+                    "tensor_frac": round(2 * flops / ((tq + tdq) * 1e-3) / 1e12 / bf16_peak, 4),
+                    "roofline": roofline_hbm(alg_quant(n) + alg_dequant(n), tq + tdq)})
+        del v, codes, norms, o
+
     if want("kv_k"):
         G, T, d, m, nq = 32, 32768, 128, 256, 32
         k = synth.kv_with_channels(4, 8, T, d, seed=3, device=dev).reshape(-1)
@@ -762,7 +788,7 @@ def profile_case(case):
         rq.rq_dequantize(codes, norms, LAYER_N, D, BITS, rq.RQ_CODES_PACKED, 1, 1000, cent, out)
     else:
         key = {"weight4096_fused": "weight4096", "kv_sketch": "kv_k", "kv_score": "kv_k", "kv_attention": "kv_k",
-               "kv_v": "kv_v", "kv_v96": "kv_v96", "tq256": "tq256", "tq512": "tq512"}[case]
+               "kv_v": "kv_v", "kv_v96": "kv_v96", "kv_dense": "kv_dense", "tq256": "tq256", "tq512": "tq512"}[case]
         secondary_lines(dev, reps=1, only=key)
     torch.cuda.synchronize()
     assert rq.rq_device_error(True) == 0

@@ -136,6 +136,48 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
                         rq_layout layout, int use_signs, uint64_t sign_seed, const float *centroids,
                         void *out, rq_dtype out_dtype, rq_stream_t stream);
 
+/* ---- Dense random orthogonal rotation with the Beta-law codebook ----------
+ * TurboQuant README, "Algorithm in one paragraph": store ||x||, rotate the
+ * unit vector x / ||x|| by a fixed random orthogonal Pi drawn by the QR
+ * decomposition of a Gaussian matrix with the sign fix, bucketize every
+ * coordinate against the Lloyd-Max centroids of the law of one coordinate of
+ * a uniform unit vector (t^2 ~ Beta(1/2, (d-1)/2)), bit-pack; the inverse is
+ * x^ = ||x|| Pi^T c.  The rotation runs as a 16-bit tensor-core GEMM with
+ * fp32 accumulation, so a code next to a boundary may differ from an exact
+ * evaluation by one level. */
+
+/* Lloyd-Max centroids of f_d(t) ~ (1 - t^2)^((d-3)/2) on [-1, 1] at `bits`
+ * (1..8), 3 <= d <= 65536, ascending, exactly odd-symmetric, written to the
+ * HOST array centroids_out[2^bits] as fp32 (a float64 fixed point: cell
+ * means by Gauss-Legendre quadrature and the closed-form first moment).
+ * Host only; well under a second up to 4 bits, about half a minute at 8. */
+rq_status rq_beta_lloyd_max(int d, int bits, float *centroids_out);
+
+/* The seeded rotation Pi (d x d, row-major fp32) into the HOST array pi_out:
+ * G[i][j] = Box-Muller normal k = i*d + j over SplitMix64(seed) outputs 2k
+ * and 2k+1 (the stream qjl_make_projection uses), Householder QR in float64,
+ * Pi = Q diag(sign(diag R)).  1 <= d <= 4096.  Host only, O(d^3). */
+rq_status rq_make_rotation(int d, uint64_t seed, float *pi_out);
+
+/* Quantize n values of x (dtype fp16/bf16, blocks of d contiguous, d = 128)
+ * with the rotation pi (DEVICE, d x d row-major, the same dtype as x):
+ *   norms[b] = fp16(||x_b||) (the canonical fp32 pairwise norm),
+ *   codes[b] = #{t_k < z_j}, z = (Pi x_b) * (1 / ||x_b||) in fp32,
+ *   t_k = fl32((c_k + c_k+1) / 2); centroids: HOST, 2^bits ascending fp32
+ *   (rq_beta_lloyd_max(d, bits) for the method's codebook).
+ * codes: rq_code_bytes(n, d, bits, layout) bytes.  All device pointers
+ * 16-byte aligned (RQ_EALIGN); other d return RQ_EUNSUPPORTED. */
+rq_status rq_quantize_dense(const void *x, rq_dtype dtype, int64_t n, int d, const void *pi, int bits,
+                            rq_layout layout, const float *centroids, void *codes, uint16_t *norms,
+                            rq_stream_t stream);
+
+/* x^_b = n16_b * Pi^T c_b into out (dtype, also the dtype of pi), where c_b
+ * holds the centroids of the codes, each rounded once to dtype (the GEMM
+ * operand), accumulated in fp32 and rounded once to dtype. */
+rq_status rq_dequantize_dense(const void *codes, const uint16_t *norms, int64_t n, int d, const void *pi, int bits,
+                              rq_layout layout, const float *centroids, void *out, rq_dtype dtype,
+                              rq_stream_t stream);
+
 /* Quantize (as rq_quantize) and sketch the first-stage residual in the same
  * pass (the optional 1-bit QJL residual correction of the PolarQuant
  * paragraph; the two-stage TurboQuant-style key code):

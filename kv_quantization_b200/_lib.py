@@ -59,6 +59,10 @@ def lib() -> C.CDLL:
                                         vp, vp, vp, i32, i32, i32, u64, vp, C.c_float, vp, vp, sz, vp]),
                 "qjl_score_noalloc": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32,
                                             u64, fp, vp, vp]),
+                "rq_beta_lloyd_max": (i32, [i32, i32, fp]),
+                "rq_make_rotation": (i32, [i32, u64, fp]),
+                "rq_quantize_dense": (i32, [vp, i32, i64, i32, vp, i32, i32, fp, vp, vp, vp]),
+                "rq_dequantize_dense": (i32, [vp, vp, i64, i32, vp, i32, i32, fp, vp, i32, vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -72,7 +76,8 @@ def exported_symbols():
     """Names this binding expects librq.so to export."""
     return ["rq_status_string", "rq_device_error", "rq_last_launch", "rq_probe_bounded_wait", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
             "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score",
-            "qjl_score_noalloc", "qjl_attention_workspace_bytes", "qjl_attention"]
+            "qjl_score_noalloc", "qjl_attention_workspace_bytes", "qjl_attention", "rq_beta_lloyd_max",
+            "rq_make_rotation", "rq_quantize_dense", "rq_dequantize_dense"]
 
 
 def status_string(status: int) -> str:
@@ -145,6 +150,33 @@ def rq_dequantize(codes, norms, n, d, bits, layout, use_signs, sign_seed, centro
     c, cp = _table(centroids)
     _check("rq_dequantize", lib().rq_dequantize(_dev(codes), _dev(norms), n, d, bits, layout, int(use_signs),
                                                 sign_seed, cp, _dev(out), _dtype_code(out), _stream(stream)))
+
+
+def rq_beta_lloyd_max(d: int, bits: int) -> np.ndarray:
+    """Lloyd-Max centroids (fp32, ascending) of one coordinate of a uniform unit vector in R^d."""
+    out = np.zeros(1 << bits, np.float32)
+    _check("rq_beta_lloyd_max", lib().rq_beta_lloyd_max(d, bits, out.ctypes.data_as(C.POINTER(C.c_float))))
+    return out
+
+
+def rq_make_rotation(d: int, seed: int) -> np.ndarray:
+    """The seeded random orthogonal matrix Pi (d x d, fp32, row-major)."""
+    out = np.zeros((d, d), np.float32)
+    _check("rq_make_rotation", lib().rq_make_rotation(d, seed, out.ctypes.data_as(C.POINTER(C.c_float))))
+    return out
+
+
+def rq_quantize_dense(x, d, pi, bits, layout, centroids, codes, norms, stream=None, n=None):
+    c, cp = _table(centroids)
+    _check("rq_quantize_dense", lib().rq_quantize_dense(_dev(x), _dtype_code(x), x.numel() if n is None else n, d,
+                                                        _dev(pi), bits, layout, cp, _dev(codes), _dev(norms),
+                                                        _stream(stream)))
+
+
+def rq_dequantize_dense(codes, norms, n, d, pi, bits, layout, centroids, out, stream=None):
+    c, cp = _table(centroids)
+    _check("rq_dequantize_dense", lib().rq_dequantize_dense(_dev(codes), _dev(norms), n, d, _dev(pi), bits, layout,
+                                                            cp, _dev(out), _dtype_code(out), _stream(stream)))
 
 
 def rq_quantize_qjl(x, d, bits, layout, use_signs, sign_seed, centroids, m, proj, codes, norms, qjl_signs,

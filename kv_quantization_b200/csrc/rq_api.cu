@@ -672,4 +672,197 @@ rq_status qjl_score(const void *q, int64_t G, int n_q, int d, int m, const void 
     return cuda_status(rq::launch_score(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------------------ dense rotation
+
+namespace {
+
+// Gauss-Legendre nodes and weights on [-1, 1]: Newton iteration on P_n from the
+// three-term recurrence (k P_k = (2k - 1) z P_{k-1} - (k - 1) P_{k-2}).
+void gauss_legendre16(double *x, double *w)
+{
+    constexpr int n = 16;
+    const double pi = 3.14159265358979323846;
+    for (int i = 0; i < n / 2; ++i) {
+        double z = std::cos(pi * (i + 0.75) / (n + 0.5)), dp = 1.0;
+        for (int it = 0; it < 100; ++it) {
+            double p0 = 1.0, p1 = z;
+            for (int k = 2; k <= n; ++k) {
+                const double p2 = ((2.0 * k - 1.0) * z * p1 - (k - 1.0) * p0) / k;
+                p0 = p1;
+                p1 = p2;
+            }
+            dp = n * (z * p1 - p0) / (z * z - 1.0);
+            const double dz = p1 / dp;
+            z -= dz;
+            if (std::fabs(dz) < 1e-16) break;
+        }
+        x[i] = -z;
+        x[n - 1 - i] = z;
+        w[i] = w[n - 1 - i] = 2.0 / ((1.0 - z * z) * dp * dp);
+    }
+}
+
+// Unnormalised mass of f_d(t) ~ (1 - t^2)^((d-3)/2) over [a, b] (0 <= a < b <= 1):
+// composite 16-point Gauss-Legendre, panels a quarter of the law's width 1/sqrt(d).
+double beta_mass(double a, double b, int d, const double *gx, const double *gw)
+{
+    const double al = 0.5 * (d - 3);
+    int panels = (int)std::ceil((b - a) * std::sqrt((double)d) * 4.0);
+    panels = panels < 4 ? 4 : (panels > 8192 ? 8192 : panels);
+    const double h = (b - a) / panels;
+    double s = 0.0;
+    for (int p = 0; p < panels; ++p) {
+        const double m = a + (p + 0.5) * h;
+        for (int k = 0; k < 16; ++k) {
+            const double t = m + 0.5 * h * gx[k];
+            s += gw[k] * (al == 0.0 ? 1.0 : std::exp(al * std::log1p(-t * t)));
+        }
+    }
+    return 0.5 * h * s;
+}
+
+// Unnormalised first moment over [a, b]: d/dt (1 - t^2)^((d-1)/2) = -(d-1) t (1 - t^2)^((d-3)/2).
+double beta_moment(double a, double b, int d)
+{
+    const double k = 0.5 * (d - 1);
+    auto g = [&](double t) { return t >= 1.0 ? 0.0 : std::exp(k * std::log1p(-t * t)); };
+    return (g(a) - g(b)) / (2.0 * k);
+}
+
+}  // namespace
+
+rq_status rq_beta_lloyd_max(int d, int bits, float *centroids_out)
+{
+    if (d < 3 || d > 65536 || bits < 1 || bits > 8 || !centroids_out) return RQ_EINVAL;
+    const int K = 1 << bits, h = K / 2;
+    double gx[16], gw[16];
+    gauss_legendre16(gx, gw);
+    std::vector<double> c(h), t(h + 1);
+    for (int k = 0; k < h; ++k) c[k] = (k + 0.5) / h * std::fmin(1.0, 3.0 / std::sqrt((double)d));
+    for (int it = 0; it < 200000; ++it) {
+        t[0] = 0.0;
+        t[h] = 1.0;
+        for (int k = 1; k < h; ++k) t[k] = 0.5 * (c[k - 1] + c[k]);
+        double worst = 0.0;
+        for (int k = 0; k < h; ++k) {
+            const double nc = beta_moment(t[k], t[k + 1], d) / beta_mass(t[k], t[k + 1], d, gx, gw);
+            worst = std::fmax(worst, std::fabs(nc - c[k]));
+            c[k] = nc;
+        }
+        if (worst < 1e-15) break;
+    }
+    for (int k = 0; k < h; ++k) {
+        centroids_out[h + k] = (float)c[k];
+        centroids_out[h - 1 - k] = (float)-c[k];
+    }
+    return RQ_OK;
+}
+
+rq_status rq_make_rotation(int d, uint64_t seed, float *pi_out)
+{
+    if (d < 1 || d > 4096 || !pi_out) return RQ_EINVAL;
+    const size_t n = (size_t)d;
+    std::vector<double> A(n * n), V(n * n, 0.0), beta(n, 0.0), rdiag(n, 0.0);
+    for (size_t i = 0; i < n; ++i)                  // G[i][j] = Box-Muller over SplitMix64 outputs 2k, 2k+1
+        for (size_t j = 0; j < n; ++j) {
+            const uint64_t k = (uint64_t)(i * n + j);
+            const double u1 = (double)((splitmix64(seed, 2ull * k) >> 11) + 1ull) * 0x1p-53;
+            const double u2 = (double)(splitmix64(seed, 2ull * k + 1ull) >> 11) * 0x1p-53;
+            A[i * n + j] = std::sqrt(-2.0 * std::log(u1)) * std::cos(6.283185307179586476925286766559 * u2);
+        }
+    // Householder QR: reflection k maps column k below the diagonal onto e_k.
+    for (size_t k = 0; k < n; ++k) {
+        double nx = 0.0;
+        for (size_t i = k; i < n; ++i) nx += A[i * n + k] * A[i * n + k];
+        nx = std::sqrt(nx);
+        const double x0 = A[k * n + k];
+        const double alpha = x0 >= 0.0 ? -nx : nx;
+        double vv = 0.0;
+        for (size_t i = k; i < n; ++i) {
+            V[i * n + k] = A[i * n + k] - (i == k ? alpha : 0.0);
+            vv += V[i * n + k] * V[i * n + k];
+        }
+        rdiag[k] = nx == 0.0 ? 0.0 : alpha;
+        if (vv == 0.0) continue;
+        beta[k] = 2.0 / vv;
+        for (size_t j = k; j < n; ++j) {
+            double s = 0.0;
+            for (size_t i = k; i < n; ++i) s += V[i * n + k] * A[i * n + j];
+            s *= beta[k];
+            for (size_t i = k; i < n; ++i) A[i * n + j] -= s * V[i * n + k];
+        }
+    }
+    // Q = H_0 H_1 ... H_{n-1} applied to the identity, from the last reflection back.
+    std::vector<double> Q(n * n, 0.0);
+    for (size_t i = 0; i < n; ++i) Q[i * n + i] = 1.0;
+    for (size_t kk = n; kk-- > 0;) {
+        if (beta[kk] == 0.0) continue;
+        for (size_t j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (size_t i = kk; i < n; ++i) s += V[i * n + kk] * Q[i * n + j];
+            s *= beta[kk];
+            for (size_t i = kk; i < n; ++i) Q[i * n + j] -= s * V[i * n + kk];
+        }
+    }
+    // sign fix: column k times sign(R_kk)
+    for (size_t i = 0; i < n; ++i)
+        for (size_t j = 0; j < n; ++j) pi_out[i * n + j] = (float)(rdiag[j] < 0.0 ? -Q[i * n + j] : Q[i * n + j]);
+    return RQ_OK;
+}
+
+static rq_status check_dense(int64_t n, int d, int bits, rq_layout layout, rq_dtype dtype)
+{
+    if (d != 128) return (d > 0 && d <= 512) ? RQ_EUNSUPPORTED : RQ_EINVAL;
+    if (bits < 1 || bits > 8) return RQ_EINVAL;
+    if (layout != RQ_CODES_PACKED && layout != RQ_CODES_INT8) return RQ_EINVAL;
+    if (dtype != RQ_F16 && dtype != RQ_BF16) return RQ_EINVAL;
+    if (n < 0 || n % d) return RQ_EINVAL;
+    if (n / d >= ((int64_t)1 << 31)) return RQ_ESIZE;   // TMA row coordinates are int32
+    return RQ_OK;
+}
+
+rq_status rq_quantize_dense(const void *x, rq_dtype dtype, int64_t n, int d, const void *pi, int bits,
+                            rq_layout layout, const float *centroids, void *codes, uint16_t *norms,
+                            rq_stream_t stream)
+{
+    rq::begin_call();
+    rq_status s = check_dense(n, d, bits, layout, dtype);
+    if (s) return s;
+    if (n == 0) return RQ_OK;
+    if (!x || !pi || !codes || !norms) return RQ_EINVAL;
+    if (!aligned16(x) || !aligned16(pi) || !aligned16(codes) || !aligned16(norms)) return RQ_EALIGN;
+    QuantTables T;
+    s = tables_for(centroids, bits, d, 0, 0, T);
+    if (s) return s;
+    rq::DenseArgs a{};
+    a.nvec = n / d; a.bf16 = dtype == RQ_BF16; a.pw = layout == RQ_CODES_INT8 ? 8 : bits; a.tables = &T;
+    a.codes = static_cast<uint8_t *>(codes); a.norms = norms; a.num_sms = num_sms();
+    if (a.num_sms <= 0) return RQ_ECUDA;
+    if (!rq::make_vectors_tmap(&a.tmap_x, x, a.nvec, d, 128) || !rq::make_proj_tmap(&a.tmap_pi, pi, d, d, 128))
+        return RQ_ECUDA;
+    return cuda_status(rq::launch_quantize_dense(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rq_status rq_dequantize_dense(const void *codes, const uint16_t *norms, int64_t n, int d, const void *pi, int bits,
+                              rq_layout layout, const float *centroids, void *out, rq_dtype dtype,
+                              rq_stream_t stream)
+{
+    rq::begin_call();
+    rq_status s = check_dense(n, d, bits, layout, dtype);
+    if (s) return s;
+    if (n == 0) return RQ_OK;
+    if (!codes || !norms || !pi || !out) return RQ_EINVAL;
+    if (!aligned16(codes) || !aligned16(norms) || !aligned16(pi) || !aligned16(out)) return RQ_EALIGN;
+    QuantTables T;
+    s = tables_for(centroids, bits, d, 0, 0, T);
+    if (s) return s;
+    rq::DenseArgs a{};
+    a.nvec = n / d; a.bf16 = dtype == RQ_BF16; a.pw = layout == RQ_CODES_INT8 ? 8 : bits; a.tables = &T;
+    a.codes_in = static_cast<const uint8_t *>(codes); a.norms_in = norms; a.out = static_cast<uint16_t *>(out);
+    a.num_sms = num_sms();
+    if (a.num_sms <= 0) return RQ_ECUDA;
+    if (!rq::make_proj_tmap(&a.tmap_pi, pi, d, d, 128)) return RQ_ECUDA;
+    return cuda_status(rq::launch_dequantize_dense(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -88,6 +88,24 @@ void note_launch(const char *kernel);
 
 cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st);
 // Blocks of a size d that is not a power of two (rq_bd.cuh): 64 < d < 512, d % 32 == 0.
+// Dense-rotation quantization (rq_dense.cuh), d = 128.
+struct DenseArgs {
+    int64_t nvec;
+    bool bf16;
+    int pw;                    // bits per stored code (8 for the int8 layout)
+    const QuantTables *tables;
+    const uint8_t *codes_in;   // dequantize
+    uint8_t *codes;            // quantize
+    uint16_t *norms;
+    const uint16_t *norms_in;
+    uint16_t *out;
+    int num_sms;
+    CUtensorMap tmap_x;        // blocks as {64, 2, nvec}, {64, 1, 128} boxes (quantize)
+    CUtensorMap tmap_pi;       // Pi as [128][128], {64, 128} boxes
+};
+cudaError_t launch_quantize_dense(const DenseArgs &a, cudaStream_t st);
+cudaError_t launch_dequantize_dense(const DenseArgs &a, cudaStream_t st);
+
 bool bd_size(int d);
 cudaError_t launch_quantize_bd(const QuantArgs &a, cudaStream_t st);
 cudaError_t launch_dequantize_bd(const DequantArgs &a, cudaStream_t st);

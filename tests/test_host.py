@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 
 import oracle as O
+import kv_quantization_b200 as rq
 from kv_quantization_b200 import _lib as L
 from tests.conftest import ROOT, read_golden
 
@@ -191,3 +192,40 @@ def test_block_diagonal_sizes_take_no_residual_sketch():
                           stream=0, n=96 * 64)
     assert e.value.status == -4
     assert L.rq_last_launch() == ""
+
+
+# ---------------------------------------------------------------- dense rotation (host tables)
+
+@pytest.mark.parametrize("d,bits", [(3, 2), (16, 1), (128, 2), (128, 4), (512, 3)])
+def test_beta_lloyd_max_matches_the_oracle(d, bits):
+    from oracle import dense_rotation as D
+    got = rq.rq_beta_lloyd_max(d, bits).astype(np.float64)
+    want = D.beta_lloyd_max(d, bits)
+    np.testing.assert_allclose(got, want.astype(np.float32).astype(np.float64), rtol=2e-7, atol=1e-9)
+    assert np.all(got[1:] > got[:-1]) and np.array_equal(got, -got[::-1])
+
+
+@pytest.mark.parametrize("d", [8, 64, 128])
+def test_make_rotation_matches_the_oracle(d):
+    from oracle import dense_rotation as D
+    got = rq.rq_make_rotation(d, 21).astype(np.float64)
+    np.testing.assert_allclose(got, D.rotation(21, d), atol=2e-7)
+
+
+def test_dense_entry_points_validate_before_launch():
+    import torch
+    x = torch.zeros(256, dtype=torch.bfloat16)
+    pi = torch.zeros(128, 128, dtype=torch.bfloat16)
+    codes = torch.zeros(128, dtype=torch.uint8)
+    norms = torch.zeros(2, dtype=torch.int16)
+    c = rq.rq_beta_lloyd_max(128, 4)
+    for d, want in ((64, "RQ_EUNSUPPORTED"), (100, "RQ_EUNSUPPORTED"), (0, "RQ_EINVAL")):
+        with pytest.raises(rq.RQError, match=want):
+            rq.rq_quantize_dense(x, d, pi, 4, rq.RQ_CODES_PACKED, c, codes, norms, stream=0)
+    with pytest.raises(rq.RQError, match="RQ_EINVAL"):
+        rq.rq_quantize_dense(x, 128, pi, 4, rq.RQ_CODES_PACKED, c, codes, norms, n=200, stream=0)
+    with pytest.raises(rq.RQError, match="RQ_EINVAL"):
+        rq.rq_dequantize_dense(codes, norms, 256, 128, pi, 9, rq.RQ_CODES_PACKED, c, x, stream=0)
+    assert L.rq_last_launch() == ""
+    with pytest.raises(rq.RQError, match="RQ_EINVAL"):
+        rq.rq_beta_lloyd_max(2, 4)
