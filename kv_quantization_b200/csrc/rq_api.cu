@@ -861,7 +861,8 @@ rq_status rq_dequantize_dense(const void *codes, const uint16_t *norms, int64_t 
     a.codes_in = static_cast<const uint8_t *>(codes); a.norms_in = norms; a.out = static_cast<uint16_t *>(out);
     a.num_sms = num_sms();
     if (a.num_sms <= 0) return RQ_ECUDA;
-    if (!rq::make_proj_tmap(&a.tmap_pi, pi, d, d, 128)) return RQ_ECUDA;
+    if (!rq::make_proj_tmap(&a.tmap_pi, pi, d, d, 128) || !rq::make_vectors_tmap(&a.tmap_out, out, a.nvec, d, 128))
+        return RQ_ECUDA;
     return cuda_status(rq::launch_dequantize_dense(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -30,8 +30,8 @@ cudaError_t run_dequantize_dense(const DenseArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const int64_t tiles = (a.nvec + 127) / 128;
     const int64_t grid = tiles < (int64_t)a.num_sms ? tiles : (int64_t)a.num_sms;
-    kern<<<(unsigned)(grid > 0 ? grid : 1), kDnDWarps * 32, smem, st>>>(a.tmap_pi, a.codes_in, a.norms_in, a.nvec,
-                                                                        *a.tables, a.out);
+    kern<<<(unsigned)(grid > 0 ? grid : 1), kDnDWarps * 32, smem, st>>>(a.tmap_pi, a.tmap_out, a.codes_in, a.norms_in,
+                                                                        a.nvec, *a.tables);
     note_launch("dequantize_dense_kernel");
     return cudaGetLastError();
 }
@@ -56,14 +56,14 @@ template <bool BF16>
 cudaError_t dequantize_dense_pw(const DenseArgs &a, cudaStream_t st)
 {
     switch (a.pw) {
-    case 1: return run_dequantize_dense<BF16, 1, 4>(a, st);
-    case 2: return run_dequantize_dense<BF16, 2, 4>(a, st);
-    case 3: return run_dequantize_dense<BF16, 3, 4>(a, st);
-    case 4: return run_dequantize_dense<BF16, 4, 4>(a, st);
-    case 5: return run_dequantize_dense<BF16, 5, 4>(a, st);
-    case 6: return run_dequantize_dense<BF16, 6, 4>(a, st);
-    case 7: return run_dequantize_dense<BF16, 7, 4>(a, st);
-    case 8: return run_dequantize_dense<BF16, 8, 4>(a, st);
+    case 1: return run_dequantize_dense<BF16, 1, 3>(a, st);
+    case 2: return run_dequantize_dense<BF16, 2, 3>(a, st);
+    case 3: return run_dequantize_dense<BF16, 3, 3>(a, st);
+    case 4: return run_dequantize_dense<BF16, 4, 3>(a, st);
+    case 5: return run_dequantize_dense<BF16, 5, 3>(a, st);
+    case 6: return run_dequantize_dense<BF16, 6, 3>(a, st);
+    case 7: return run_dequantize_dense<BF16, 7, 3>(a, st);
+    case 8: return run_dequantize_dense<BF16, 8, 3>(a, st);
     default: return cudaErrorNotSupported;
     }
 }

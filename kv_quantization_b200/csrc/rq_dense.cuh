@@ -25,7 +25,8 @@
 //             the K-major A operand C of the tile;
 //   warp 4    MMA: X^ = C Pi (B = Pi read MN-major: row j of Pi is K step j,
 //             its columns the 128 outputs) into one of two TMEM buffers;
-//   warps 5-12 epilogue: x^ = acc * n16, rounded to the output dtype, stored.
+//   warps 5-12 epilogue: x^ = acc * n16, rounded to the output dtype, staged
+//             in the swizzled output layout, stored by TMA.
 // Pi stays in shared memory for the CTA's whole run.  Every wait is bounded
 // (mbar_wait); an expired wait sets the device error word and the roles stop.
 #pragma once
@@ -53,6 +54,11 @@ __device__ __forceinline__ uint64_t dense_desc_sw128(uint32_t saddr, uint32_t lb
     d |= (uint64_t)1 << 46;
     d |= (uint64_t)2 << 61;
     return d;
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __host__ __device__ inline size_t quantize_dense_smem(int stages, int lut_cells)
@@ -242,14 +248,14 @@ quantize_dense_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_cons
 __host__ __device__ inline size_t dequantize_dense_smem(int stages, int pw)
 {
     const size_t tab = pw <= 4 ? ((size_t)1 << (2 * pw)) * 16 * 4 : 256 * 2;
-    return 1024 + kDnTile + (size_t)stages * kDnTile + tab + 8 * (2 * stages + 8) + 16;
+    return 1024 + 2 * kDnTile + (size_t)stages * kDnTile + tab + 8 * (2 * stages + 8) + 16;
 }
 
 template <bool BF16, int PW, int NS>
 __global__ void __launch_bounds__(kDnDWarps * 32, 1)
-dequantize_dense_kernel(const __grid_constant__ CUtensorMap tmp, const uint8_t *__restrict__ codes,
-                        const uint16_t *__restrict__ norms, int64_t nvec, const __grid_constant__ QuantTables T,
-                        uint16_t *__restrict__ out)
+dequantize_dense_kernel(const __grid_constant__ CUtensorMap tmp, const __grid_constant__ CUtensorMap tmo,
+                        const uint8_t *__restrict__ codes, const uint16_t *__restrict__ norms, int64_t nvec,
+                        const __grid_constant__ QuantTables T)
 {
     constexpr int CB = 16 * PW;
     constexpr bool kPairs = PW <= 4;
@@ -257,7 +263,8 @@ dequantize_dense_kernel(const __grid_constant__ CUtensorMap tmp, const uint8_t *
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *s_P = base;                                    // Pi rows (K) x two 64-wide column atoms (N)
-    uint8_t *ring = s_P + kDnTile;                          // A stages: C, K-major
+    uint8_t *s_O = s_P + kDnTile;                           // output tile staged for the TMA store
+    uint8_t *ring = s_O + kDnTile;                          // A stages: C, K-major
     uint32_t *ptab = reinterpret_cast<uint32_t *>(ring + (size_t)NS * kDnTile);   // pairs x 16 copies
     uint16_t *ctab = reinterpret_cast<uint16_t *>(ptab);                          // or single levels
     const size_t tab_bytes = kPairs ? (size_t)NE * 16 * 4 : 256 * 2;
@@ -296,6 +303,7 @@ dequantize_dense_kernel(const __grid_constant__ CUtensorMap tmp, const uint8_t *
         mbar_init(&p_ready[0], 1);
         fence_barrier_init();
         prefetch_tmap(&tmp);
+        prefetch_tmap(&tmo);
         mbar_arrive_expect_tx(&p_ready[0], kDnTile);
         for (int kc = 0; kc < 2; ++kc) tma_load_2d(s_P + (size_t)kc * 16384, &tmp, 64 * kc, 0, &p_ready[0]);
     }
@@ -310,17 +318,25 @@ dequantize_dense_kernel(const __grid_constant__ CUtensorMap tmp, const uint8_t *
         // ------------------------------------------------------------ producers: C tile
         const int r = tid;                                  // block within the tile
         const uint32_t ptab_lane = smem_u32(ptab) + (uint32_t)(lane & 15) * 4u;
-        for (int64_t i = 0; i < my_tiles && ok; ++i) {
-            const int s = (int)(i % NS);
-            const int64_t use = i / NS;
+        // the codes of tile i + 1 are loaded while tile i is unpacked
+        auto load_codes = [&](int64_t i, uint32_t *w) {
             const int64_t tok = (blockIdx.x + i * gridDim.x) * 128 + r;
-            uint32_t w[4 * PW];
-            if (tok < nvec) {
+            if (i < my_tiles && tok < nvec) {
                 load_bytes<CB>(codes + tok * CB, w);
             } else {
 #pragma unroll
                 for (int k = 0; k < 4 * PW; ++k) w[k] = 0u;
             }
+        };
+        uint32_t wn[4 * PW];
+        load_codes(0, wn);
+        for (int64_t i = 0; i < my_tiles && ok; ++i) {
+            const int s = (int)(i % NS);
+            const int64_t use = i / NS;
+            uint32_t w[4 * PW];
+#pragma unroll
+            for (int k = 0; k < 4 * PW; ++k) w[k] = wn[k];
+            load_codes(i + 1, wn);
             if (use > 0 && !mbar_wait(&a_free[s], (uint32_t)((use - 1) & 1))) { ok = false; break; }
             const uint32_t A = smem_u32(ring + (size_t)s * kDnTile);
 #pragma unroll
@@ -371,36 +387,63 @@ dequantize_dense_kernel(const __grid_constant__ CUtensorMap tmp, const uint8_t *
         }
     } else {
         // ------------------------------------------------------------ epilogue: x^ = acc * n16
+        // The 8 warps stage the tile in s_O (the TMA layout of the output:
+        // two 64-column regions, 128-byte swizzle) and one thread stores it.
+        // Every warp takes both named barriers of every tile, also after an
+        // expired wait (it then skips the work), so none can wait forever.
         const int quarter = warp & 3;
         const int part = (warp - 5) >> 2;                   // chunks 2 part, 2 part + 1
-        for (int64_t i = 0; i < my_tiles && ok; ++i) {
+        const bool leader = warp == 5 && lane == 0;
+        const uint32_t sO = smem_u32(s_O);
+        for (int64_t i = 0; i < my_tiles; ++i) {
             const int a = (int)(i & 1);
             const int row = quarter * 32 + lane;
-            const int64_t tok = (blockIdx.x + i * gridDim.x) * 128 + row;
+            const int64_t t = blockIdx.x + i * gridDim.x;
+            const int64_t tok = t * 128 + row;
             const float n16 = tok < nvec ? h16_to_f32(__ldg(norms + tok)) : 0.0f;
-            if (!mbar_wait(&acc_full[a], (uint32_t)((i >> 1) & 1))) { ok = false; break; }
+            if (ok && !mbar_wait(&acc_full[a], (uint32_t)((i >> 1) & 1))) ok = false;
             tc_fence_after();
             uint32_t acc[2][32];
+            if (ok) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
-                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 128 + 32 * (2 * part + q)), acc[q]);
-            tmem_ld_wait();
+                for (int q = 0; q < 2; ++q)
+                    tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 128 + 32 * (2 * part + q)), acc[q]);
+                tmem_ld_wait();
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cta(&acc_free[a]);
-            const float2 n2 = make_float2(n16, n16);
+            if (lane == 0 && ok) mbar_arrive_cta(&acc_free[a]);
+            if (leader) bulk_wait_read<0>();                 // the previous tile's store has read s_O
+            named_barrier_sync(1, 256);
+            if (ok) {
+                const float2 n2 = make_float2(n16, n16);
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                uint32_t o[16];
+                for (int q = 0; q < 2; ++q) {
+                    const int col0 = 32 * (2 * part + q);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float2 v = __fmul2_rn(make_float2(__uint_as_float(acc[q][2 * j]), __uint_as_float(acc[q][2 * j + 1])),
-                                                n2);
-                    o[j] = pack2<BF16>(v.x, v.y);
+                    for (int c8 = 0; c8 < 4; ++c8) {        // 8 values = one 16-byte chunk of the row
+                        uint32_t o[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int e = 8 * c8 + 2 * j;
+                            const float2 v = __fmul2_rn(make_float2(__uint_as_float(acc[q][e]), __uint_as_float(acc[q][e + 1])), n2);
+                            o[j] = pack2<BF16>(v.x, v.y);
+                        }
+                        const int col = col0 + 8 * c8;
+                        sts128(sO + (uint32_t)(col >> 6) * 16384u + sw128_offset(row, (col & 63) >> 3),
+                               make_uint4(o[0], o[1], o[2], o[3]));
+                    }
                 }
-                if (tok < nvec) store_bytes<64>(reinterpret_cast<uint8_t *>(out + tok * 128 + 32 * (2 * part + q)), o);
+            }
+            fence_proxy_async_smem();                       // generic writes -> visible to the TMA store
+            named_barrier_sync(1, 256);
+            if (leader && ok) {
+                tma_store_3d(&tmo, 0, 0, (int)(t * 128), s_O);
+                tma_store_3d(&tmo, 0, 1, (int)(t * 128), s_O + 16384);
+                bulk_commit();
             }
         }
+        if (leader) bulk_wait<0>();
     }
     tc_fence_before();
     __syncthreads();

@@ -102,6 +102,7 @@ struct DenseArgs {
     int num_sms;
     CUtensorMap tmap_x;        // blocks as {64, 2, nvec}, {64, 1, 128} boxes (quantize)
     CUtensorMap tmap_pi;       // Pi as [128][128], {64, 128} boxes
+    CUtensorMap tmap_out;      // output blocks as {64, 2, nvec}, {64, 1, 128} boxes (dequantize)
 };
 cudaError_t launch_quantize_dense(const DenseArgs &a, cudaStream_t st);
 cudaError_t launch_dequantize_dense(const DenseArgs &a, cudaStream_t st);
