@@ -720,6 +720,22 @@ def cpu_baseline():
     O.attention(q16, 1, 32, 128, 256, S, O.BF16, sg[: 2048 * 32], kn[:2048], 2048, vcd, vnr, 4, O.PACKED, vs, c4,
                 1.0 / 128 ** 0.5)
     pw["kv_attention_token_heads_per_s"] = round(2048 / (time.perf_counter() - t0), 1)
+    # V cache at head dim 96 (block-diagonal transform): 16384 blocks round trip
+    v96 = synth.as_u16(synth.kv_with_channels(1, 1, 16384, 96, seed=13, device="cpu")).reshape(-1)
+    s96 = O.sign_diagonal(14, 96)
+    t0 = time.perf_counter()
+    cds, nrm, _, _ = O.quantize(v96, O.BF16, 96, 4, O.PACKED, s96, c4)
+    O.dequantize(cds, nrm, 96, 4, O.PACKED, s96, c4, O.BF16)
+    pw["kv_v96_round_trip_gbs"] = round(v96.size * 2 / (time.perf_counter() - t0) / 1e9, 6)
+    # V cache with the dense rotation and the Beta codebook: 16384 blocks round trip (numpy fp64)
+    from oracle import dense_rotation as DR
+    pi16 = DR.to16(DR.rotation(17, 128), O.BF16)
+    cb = DR.beta_lloyd_max(128, 4).astype(np.float32)
+    vd = synth.as_u16(synth.kv_with_channels(1, 1, 16384, 128, seed=13, device="cpu")).reshape(-1)
+    t0 = time.perf_counter()
+    cds, nrm, _, _ = DR.quantize(vd, O.BF16, 128, pi16, 4, O.PACKED, cb)
+    DR.dequantize(cds, nrm, 16384, 128, pi16, 4, O.PACKED, DR.to16(cb, O.BF16), O.BF16, O.BF16)
+    pw["kv_dense_round_trip_gbs"] = round(vd.size * 2 / (time.perf_counter() - t0) / 1e9, 6)
     # TurboQuant-style keys at d = 256 / 512: compress 2048 keys, score 32 queries over 2048 keys
     for d in (256, 512):
         kk = synth.normal((1, 2048, d), seed=6, device="cpu").reshape(-1)
