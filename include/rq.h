@@ -136,6 +136,47 @@ rq_status rq_dequantize(const void *codes, const uint16_t *norms, int64_t n, int
                         rq_layout layout, int use_signs, uint64_t sign_seed, const float *centroids,
                         void *out, rq_dtype out_dtype, rq_stream_t stream);
 
+/* ---- QJL key sketch with a per-group outlier sketch ------------------------
+ * QJL README, "Algorithm in one paragraph" (outlier coordinates get a top-k
+ * sketch per group of group_size consecutive tokens, with its own projection
+ * dimension), and qjl_apply.py's key hook (per group, the norm of every
+ * coordinate over the group's tokens; the top outlier_count of them as uint8
+ * indices; one projection and the outlier dimension handed to the quantizer).
+ * Groups are 32 consecutive key vectors (a head's token count must be a
+ * multiple of 32).  Per group the outlier set O = the n_out coordinates with
+ * the largest fp32 sum of squares over the group's tokens (summed in token
+ * order; ties to the lower coordinate), stored largest first.  Each key splits
+ * into k_in (O zeroed) and k_out (only O):
+ *   signs / norms          = sign bits of S k_in and fp16(||k_in||) (as qjl_sketch);
+ *   out_signs / out_norms  = sign bits of S_o k_out, S_o = rows 0 .. m_o-1 of S,
+ *                            and fp16(||k_out||) (fp32 squares in stored order);
+ * and the score is  sqrt(pi/2)/m ||k_in|| <S q, sign(S k_in)>
+ *                 + sqrt(pi/2)/m_o ||k_out|| <S_o q_O, sign(S_o k_out)>,
+ * q_O the query on O: the sum of the two QJL estimators of <q, k_in> and
+ * <q, k_out>, unbiased for <q, k>. */
+
+/* Bytes of scratch qjl_sketch_outlier needs: the masked keys (n_vec * d bf16). */
+size_t qjl_sketch_outlier_workspace_bytes(int64_t n_vec, int d);
+
+/* keys: bf16 [n_vec][d], n_vec % 32 == 0, d = 128 (other powers of two:
+ * RQ_EUNSUPPORTED); proj: bf16 [m][d], m % 8 == 0, 8 <= m <= 512; 32 <= m_o <=
+ * min(m, 256), m_o % 32 == 0; 1 <= n_out <= 16.  Outputs (device, 16-byte
+ * aligned): signs [n_vec][m/8], norms [n_vec] fp16, out_idx [n_vec/32][n_out]
+ * uint8, out_signs [n_vec][m_o/8], out_norms [n_vec] fp16.  Sign bit = (P >= 0),
+ * bit j of byte b <-> coordinate 8b + j. */
+rq_status qjl_sketch_outlier(const void *keys, int64_t n_vec, int d, int m, const void *proj, int m_o, int n_out,
+                             uint8_t *signs, uint16_t *norms, uint8_t *out_idx, uint8_t *out_signs,
+                             uint16_t *out_norms, void *workspace, size_t workspace_bytes, rq_stream_t stream);
+
+/* Scores [G][n_q][T] (fp32) of bf16 queries q [G][n_q][d] against G * T keys
+ * sketched by qjl_sketch_outlier (T % 32 == 0; the same m, m_o, n_out, proj):
+ * the pure-QJL score of the main sketch (qjl_score) plus the outlier term.
+ * workspace: qjl_score_workspace_bytes(G, n_q, d, m). */
+rq_status qjl_score_outlier(const void *q, int64_t G, int n_q, int d, int m, const void *proj, const uint8_t *signs,
+                            const uint16_t *norms, int64_t T, int m_o, int n_out, const uint8_t *out_idx,
+                            const uint8_t *out_signs, const uint16_t *out_norms, float *scores, void *workspace,
+                            size_t workspace_bytes, rq_stream_t stream);
+
 /* ---- Dense random orthogonal rotation with the Beta-law codebook ----------
  * TurboQuant README, "Algorithm in one paragraph": store ||x||, rotate the
  * unit vector x / ||x|| by a fixed random orthogonal Pi drawn by the QR

@@ -59,6 +59,10 @@ def lib() -> C.CDLL:
                                         vp, vp, vp, i32, i32, i32, u64, vp, C.c_float, vp, vp, sz, vp]),
                 "qjl_score_noalloc": (i32, [vp, i64, i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, i32, i32, i32,
                                             u64, fp, vp, vp]),
+                "qjl_sketch_outlier_workspace_bytes": (sz, [i64, i32]),
+                "qjl_sketch_outlier": (i32, [vp, i64, i32, i32, vp, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+                "qjl_score_outlier": (i32, [vp, i64, i32, i32, i32, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, sz,
+                                            vp]),
                 "rq_beta_lloyd_max": (i32, [i32, i32, fp]),
                 "rq_make_rotation": (i32, [i32, u64, fp]),
                 "rq_quantize_dense": (i32, [vp, i32, i64, i32, vp, i32, i32, fp, vp, vp, vp]),
@@ -77,7 +81,8 @@ def exported_symbols():
     return ["rq_status_string", "rq_device_error", "rq_last_launch", "rq_probe_bounded_wait", "rq_code_bytes", "rq_lloyd_max", "rq_quantize", "rq_dequantize",
             "rq_quantize_qjl", "qjl_make_projection", "qjl_sketch", "qjl_score_workspace_bytes", "qjl_score",
             "qjl_score_noalloc", "qjl_attention_workspace_bytes", "qjl_attention", "rq_beta_lloyd_max",
-            "rq_make_rotation", "rq_quantize_dense", "rq_dequantize_dense"]
+            "rq_make_rotation", "rq_quantize_dense", "rq_dequantize_dense", "qjl_sketch_outlier_workspace_bytes",
+            "qjl_sketch_outlier", "qjl_score_outlier"]
 
 
 def status_string(status: int) -> str:
@@ -150,6 +155,26 @@ def rq_dequantize(codes, norms, n, d, bits, layout, use_signs, sign_seed, centro
     c, cp = _table(centroids)
     _check("rq_dequantize", lib().rq_dequantize(_dev(codes), _dev(norms), n, d, bits, layout, int(use_signs),
                                                 sign_seed, cp, _dev(out), _dtype_code(out), _stream(stream)))
+
+
+def qjl_sketch_outlier_workspace_bytes(n_vec: int, d: int) -> int:
+    return lib().qjl_sketch_outlier_workspace_bytes(n_vec, d)
+
+
+def qjl_sketch_outlier(keys, d, m, proj, m_o, n_out, signs, norms, out_idx, out_signs, out_norms, workspace,
+                       stream=None, n_vec=None):
+    nv = keys.numel() // d if n_vec is None else n_vec
+    _check("qjl_sketch_outlier", lib().qjl_sketch_outlier(
+        _dev(keys), nv, d, m, _dev(proj), m_o, n_out, _dev(signs), _dev(norms), _dev(out_idx), _dev(out_signs),
+        _dev(out_norms), _dev(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def qjl_score_outlier(q, G, n_q, d, m, proj, signs, norms, T, m_o, n_out, out_idx, out_signs, out_norms, scores,
+                      workspace, stream=None):
+    _check("qjl_score_outlier", lib().qjl_score_outlier(
+        _dev(q), G, n_q, d, m, _dev(proj), _dev(signs), _dev(norms), T, m_o, n_out, _dev(out_idx), _dev(out_signs),
+        _dev(out_norms), _dev(scores), _dev(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
 
 
 def rq_beta_lloyd_max(d: int, bits: int) -> np.ndarray:

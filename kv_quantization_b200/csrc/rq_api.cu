@@ -866,4 +866,72 @@ rq_status rq_dequantize_dense(const void *codes, const uint16_t *norms, int64_t 
     return cuda_status(rq::launch_dequantize_dense(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------------------ outlier sketch
+
+size_t qjl_sketch_outlier_workspace_bytes(int64_t n_vec, int d)
+{
+    return n_vec > 0 && d > 0 ? (size_t)n_vec * (size_t)d * 2 : 0;
+}
+
+static rq_status check_outlier(int d, int m, int m_o, int n_out)
+{
+    if (d != 128) return pow2_d(d) ? RQ_EUNSUPPORTED : RQ_EINVAL;
+    if (m < 8 || m > 512 || m % 8) return RQ_EINVAL;
+    if (n_out < 1 || n_out > 16 || m_o < 32 || m_o > m || m_o % 32) return RQ_EINVAL;
+    if (m_o > 256) return RQ_EUNSUPPORTED;
+    return RQ_OK;
+}
+
+rq_status qjl_sketch_outlier(const void *keys, int64_t n_vec, int d, int m, const void *proj, int m_o, int n_out,
+                             uint8_t *signs, uint16_t *norms, uint8_t *out_idx, uint8_t *out_signs,
+                             uint16_t *out_norms, void *workspace, size_t workspace_bytes, rq_stream_t stream)
+{
+    rq::begin_call();
+    rq_status s = check_outlier(d, m, m_o, n_out);
+    if (s) return s;
+    if (n_vec < 0 || n_vec % 32) return RQ_EINVAL;
+    if (n_vec > ((int64_t)1 << 34)) return RQ_ESIZE;
+    if (n_vec == 0) return RQ_OK;
+    if (!keys || !proj || !signs || !norms || !out_idx || !out_signs || !out_norms || !workspace) return RQ_EINVAL;
+    if (workspace_bytes < qjl_sketch_outlier_workspace_bytes(n_vec, d)) return RQ_ESIZE;
+    if (!aligned16(keys) || !aligned16(proj) || !aligned16(signs) || !aligned16(norms) || !aligned16(out_idx) ||
+        !aligned16(out_signs) || !aligned16(out_norms) || !aligned16(workspace))
+        return RQ_EALIGN;
+    const int sms = num_sms();
+    if (sms <= 0) return RQ_ECUDA;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = rq::launch_outlier_prep(static_cast<const uint16_t *>(keys), n_vec, n_out, m_o,
+                                            static_cast<const uint16_t *>(proj), static_cast<uint16_t *>(workspace),
+                                            out_idx, out_signs, out_norms, sms, st);
+    if (e != cudaSuccess) return RQ_ECUDA;
+    // the main sketch of the masked keys (the same checks have passed above)
+    s = qjl_sketch(workspace, RQ_BF16, n_vec, d, m, proj, signs, norms, stream);
+    rq::note_launch("outlier_prep_kernel");
+    return s;
+}
+
+rq_status qjl_score_outlier(const void *q, int64_t G, int n_q, int d, int m, const void *proj, const uint8_t *signs,
+                            const uint16_t *norms, int64_t T, int m_o, int n_out, const uint8_t *out_idx,
+                            const uint8_t *out_signs, const uint16_t *out_norms, float *scores, void *workspace,
+                            size_t workspace_bytes, rq_stream_t stream)
+{
+    rq::begin_call();
+    rq_status s = check_outlier(d, m, m_o, n_out);
+    if (s) return s;
+    if (G < 0 || n_q < 0 || T < 0 || T % 32) return RQ_EINVAL;
+    if (G > 65535 || n_q > 32 * 65535 || T > ((int64_t)1 << 31) || G * (T / 32) >= ((int64_t)1 << 31)) return RQ_ESIZE;
+    if (G == 0 || n_q == 0 || T == 0) return RQ_OK;
+    if (!q || !proj || !signs || !norms || !out_idx || !out_signs || !out_norms || !scores || !workspace)
+        return RQ_EINVAL;
+    if (workspace_bytes < rq::score_workspace_bytes(G, n_q, d, m)) return RQ_ESIZE;
+    if (!aligned16(out_idx) || !aligned16(out_signs) || !aligned16(out_norms)) return RQ_EALIGN;
+    s = qjl_score(q, G, n_q, d, m, proj, RQ_BF16, signs, norms, T, nullptr, nullptr, 0, RQ_CODES_PACKED, 0, 0,
+                  nullptr, scores, workspace, workspace_bytes, stream);
+    if (s) return s;
+    cudaError_t e = rq::launch_outlier_score(static_cast<const uint16_t *>(q), G, n_q, T, m_o, n_out,
+                                             static_cast<const uint16_t *>(proj), out_idx, out_signs, out_norms,
+                                             scores, reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status(e);
+}
+
 }  // extern "C"

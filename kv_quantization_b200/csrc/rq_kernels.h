@@ -107,6 +107,14 @@ struct DenseArgs {
 cudaError_t launch_quantize_dense(const DenseArgs &a, cudaStream_t st);
 cudaError_t launch_dequantize_dense(const DenseArgs &a, cudaStream_t st);
 
+// QJL outlier sketch (rq_outlier.cu), d = 128, groups of 32 consecutive vectors.
+cudaError_t launch_outlier_prep(const uint16_t *keys, int64_t nvec, int n_out, int m_o, const uint16_t *S,
+                                uint16_t *kin, uint8_t *idx, uint8_t *out_signs, uint16_t *out_norms, int num_sms,
+                                cudaStream_t st);
+cudaError_t launch_outlier_score(const uint16_t *q, int64_t G, int nq, int64_t T, int m_o, int n_out,
+                                 const uint16_t *S, const uint8_t *idx, const uint8_t *out_signs,
+                                 const uint16_t *out_norms, float *scores, cudaStream_t st);
+
 bool bd_size(int d);
 cudaError_t launch_quantize_bd(const QuantArgs &a, cudaStream_t st);
 cudaError_t launch_dequantize_bd(const DequantArgs &a, cudaStream_t st);

@@ -1,0 +1,214 @@
+// rq_outlier.cu -- the QJL key sketch's per-group outlier part (sm_100a).
+//
+// QJL README, "Algorithm in one paragraph", and qjl_apply.py's key hook: per
+// group of 32 consecutive tokens the top-k coordinates by their norm over the
+// group are outliers; they get their own sketch, with its own norm.  The key
+// splits into k_in (outlier coordinates zeroed) and k_out (only those):
+//   main sketch    sign(S k_in), ||k_in||   (the tensor-core key sketch, run
+//                                            on the masked keys this file writes)
+//   outlier sketch sign(S_o k_out), ||k_out||, S_o = rows 0 .. m_o-1 of S
+// and the score adds, per token, sqrt(pi/2)/m_o ||k_out|| <S_o q_O, sign(S_o k_out)>
+// with q_O the query on the group's outlier coordinates.
+//
+// outlier_prep_kernel: one warp per group.  The group's 32 keys are staged in
+//   shared memory; lane l sums the squares of columns 4l .. 4l+3 over the 32
+//   tokens in token order (fp32); the top k are taken by k rounds of a warp
+//   argmax (largest sum, ties to the lower index); then lane t (a token) reads
+//   its k outlier values, forms ||k_out|| (fp32 squares in stored order) and
+//   the m_o sign bits of sum_r S[i][O_r] v_r (fp32, stored order), and the warp
+//   writes the masked group back contiguously.
+// outlier_score_kernel: one CTA per (head, group): u[q][i] = sum_r S[i][O_r]
+//   q[O_r] for every query, then lane = token adds
+//   sqrt(pi/2)/m_o * n_out16 * sum_i u[q][i] (+1 / -1 by the sign bit) to the
+//   scores the pure-QJL score wrote.
+#include <cmath>
+#include <cstdint>
+
+#include "rq_common.cuh"
+#include "rq_kernels.h"
+
+namespace rq {
+
+namespace {
+
+constexpr int kOlWarps = 4;                 // groups per CTA (prep)
+constexpr int kOlMaxOut = 16;
+constexpr int kOlMaxMo = 256;
+
+__device__ __forceinline__ float bf16_at(const uint16_t *p) { return __uint_as_float((uint32_t)*p << 16); }
+
+__global__ void __launch_bounds__(kOlWarps * 32)
+outlier_prep_kernel(const uint16_t *__restrict__ keys, int64_t ngroups, int n_out, int m_o,
+                    const uint16_t *__restrict__ S, uint16_t *__restrict__ kin, uint8_t *__restrict__ idx_out,
+                    uint8_t *__restrict__ out_signs, uint16_t *__restrict__ out_norms)
+{
+    constexpr int d = 128;
+    extern __shared__ __align__(16) uint8_t ol_prep_smem[];
+    __shared__ int sel[kOlWarps][kOlMaxOut];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // per warp: the group's keys (8 KB), then S[i][O_r] for i < m_o (m_o * n_out floats)
+    uint8_t *wb = ol_prep_smem + (size_t)warp * (32 * d * 2 + (size_t)m_o * n_out * 4);
+    uint16_t *tl = reinterpret_cast<uint16_t *>(wb);
+    float *sow = reinterpret_cast<float *>(wb + 32 * d * 2);
+    for (int64_t g = (int64_t)blockIdx.x * kOlWarps + warp; g < ngroups; g += (int64_t)gridDim.x * kOlWarps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(keys + g * 32 * d);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) reinterpret_cast<uint4 *>(tl)[lane + 32 * i] = __ldg(src + lane + 32 * i);
+        __syncwarp();
+        // column sums of squares, token order
+        float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int t = 0; t < 32; ++t)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = bf16_at(tl + t * d + 4 * lane + c);
+                cs[c] = __fadd_rn(cs[c], __fmul_rn(v, v));
+            }
+        // top n_out: largest sum first, ties to the lower column
+        uint32_t taken = 0u;
+        for (int r = 0; r < n_out; ++r) {
+            float bv = -1.0f;
+            int bi = 1 << 30;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (!((taken >> c) & 1u) && cs[c] > bv) { bv = cs[c]; bi = 4 * lane + c; }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if ((bi >> 2) == lane) taken |= 1u << (bi & 3);
+            if (lane == 0) {
+                sel[warp][r] = bi;
+                idx_out[g * n_out + r] = (uint8_t)bi;
+            }
+        }
+        __syncwarp();
+        // S columns of the outlier set
+        for (int e = lane; e < m_o * n_out; e += 32) {
+            const int i = e / n_out, r = e - i * n_out;
+            sow[e] = bf16_at(S + (int64_t)i * d + sel[warp][r]);
+        }
+        // lane = token: outlier values, norm, sketch
+        float v[kOlMaxOut];
+        float acc = 0.0f;
+#pragma unroll
+        for (int r = 0; r < kOlMaxOut; ++r) {
+            v[r] = r < n_out ? bf16_at(tl + lane * d + sel[warp][r]) : 0.0f;
+            if (r < n_out) acc = __fadd_rn(acc, __fmul_rn(v[r], v[r]));
+        }
+        const int64_t tok = g * 32 + lane;
+        out_norms[tok] = norm_to_h16(__fsqrt_rn(acc));
+        __syncwarp();
+        for (int w = 0; w < m_o / 32; ++w) {
+            uint32_t bits = 0u;
+            for (int b = 0; b < 32; ++b) {
+                const float *row = sow + (32 * w + b) * n_out;
+                float p = 0.0f;
+#pragma unroll
+                for (int r = 0; r < kOlMaxOut; ++r)
+                    if (r < n_out) p = __fadd_rn(p, __fmul_rn(row[r], v[r]));
+                bits |= (p >= 0.0f ? 1u : 0u) << b;
+            }
+            reinterpret_cast<uint32_t *>(out_signs + tok * (m_o / 8))[w] = bits;
+        }
+        // masked group back, contiguous
+        __syncwarp();
+        for (int r = 0; r < n_out; ++r) tl[lane * d + sel[warp][r]] = 0;
+        __syncwarp();
+        uint4 *dst = reinterpret_cast<uint4 *>(kin + g * 32 * d);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[lane + 32 * i] = reinterpret_cast<const uint4 *>(tl)[lane + 32 * i];
+    }
+}
+
+__global__ void __launch_bounds__(128)
+outlier_score_kernel(const uint16_t *__restrict__ q, int nq, int64_t T, int m_o, int n_out,
+                     const uint16_t *__restrict__ S, const uint8_t *__restrict__ idx,
+                     const uint8_t *__restrict__ out_signs, const uint16_t *__restrict__ out_norms,
+                     float *__restrict__ scores)
+{
+    constexpr int d = 128;
+    extern __shared__ float ol_smem[];
+    float *u = ol_smem;                                  // [nq][m_o]
+    __shared__ float so[kOlMaxMo * kOlMaxOut];
+    __shared__ float qo[32 * kOlMaxOut];
+    __shared__ int sel[kOlMaxOut];
+    const int64_t ng = T / 32;
+    const int64_t hg = blockIdx.x;                       // (head, group)
+    const int64_t g = hg / ng, j = hg - g * ng;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid < n_out) sel[tid] = idx[hg * n_out + tid];
+    __syncthreads();
+    for (int e = tid; e < m_o * n_out; e += blockDim.x) so[e] = bf16_at(S + (int64_t)(e / n_out) * d + sel[e % n_out]);
+    const float c = (float)(1.2533141373155002512 / (double)m_o);   // sqrt(pi/2) / m_o
+    for (int q0 = 0; q0 < nq; q0 += 32) {
+        const int nqc = nq - q0 < 32 ? nq - q0 : 32;
+        __syncthreads();
+        for (int e = tid; e < nqc * n_out; e += blockDim.x) {
+            const int qq = e / n_out, r = e - qq * n_out;
+            qo[e] = bf16_at(q + (g * nq + q0 + qq) * d + sel[r]);
+        }
+        __syncthreads();
+        for (int e = tid; e < nqc * m_o; e += blockDim.x) {
+            const int qq = e / m_o, i = e - qq * m_o;
+            float s = 0.0f;
+            for (int r = 0; r < n_out; ++r) s = __fadd_rn(s, __fmul_rn(so[i * n_out + r], qo[qq * n_out + r]));
+            u[e] = s;
+        }
+        __syncthreads();
+        // lane = token of the group, warps stride over the queries
+        const int64_t tok = g * T + j * 32 + lane;
+        const float no = h16_to_f32(out_norms[tok]) * c;
+        const uint8_t *sg = out_signs + tok * (m_o / 8);
+        for (int qq = warp; qq < nqc; qq += blockDim.x / 32) {
+            const float *uq = u + qq * m_o;
+            float dot = 0.0f;
+            for (int i = 0; i < m_o; i += 8) {
+                const uint32_t byte = sg[i / 8];
+#pragma unroll
+                for (int b = 0; b < 8; ++b) dot = __fadd_rn(dot, ((byte >> b) & 1u) ? uq[i + b] : -uq[i + b]);
+            }
+            float *dst = scores + (g * nq + q0 + qq) * T + j * 32 + lane;
+            *dst = __fadd_rn(*dst, __fmul_rn(no, dot));
+        }
+    }
+}
+
+}  // namespace
+
+size_t outlier_score_smem(int nq, int m_o) { return (size_t)(nq < 32 ? nq : 32) * m_o * 4; }
+
+cudaError_t launch_outlier_prep(const uint16_t *keys, int64_t nvec, int n_out, int m_o, const uint16_t *S,
+                                uint16_t *kin, uint8_t *idx, uint8_t *out_signs, uint16_t *out_norms, int num_sms,
+                                cudaStream_t st)
+{
+    const int64_t ngroups = nvec / 32;
+    int64_t grid = (ngroups + kOlWarps - 1) / kOlWarps;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (grid > cap) grid = cap;
+    const size_t smem = (size_t)kOlWarps * (32 * 128 * 2 + (size_t)m_o * n_out * 4);
+    cudaError_t e = cudaFuncSetAttribute(outlier_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    outlier_prep_kernel<<<(unsigned)(grid > 0 ? grid : 1), kOlWarps * 32, smem, st>>>(keys, ngroups, n_out, m_o, S,
+                                                                                     kin, idx, out_signs, out_norms);
+    note_launch("outlier_prep_kernel");
+    return cudaGetLastError();
+}
+
+cudaError_t launch_outlier_score(const uint16_t *q, int64_t G, int nq, int64_t T, int m_o, int n_out,
+                                 const uint16_t *S, const uint8_t *idx, const uint8_t *out_signs,
+                                 const uint16_t *out_norms, float *scores, cudaStream_t st)
+{
+    const size_t smem = outlier_score_smem(nq, m_o);
+    cudaError_t e = cudaFuncSetAttribute(outlier_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = G * (T / 32);
+    outlier_score_kernel<<<(unsigned)blocks, 128, smem, st>>>(q, nq, T, m_o, n_out, S, idx, out_signs, out_norms,
+                                                             scores);
+    note_launch("outlier_score_kernel");
+    return cudaGetLastError();
+}
+
+}  // namespace rq

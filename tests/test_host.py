@@ -229,3 +229,26 @@ def test_dense_entry_points_validate_before_launch():
     assert L.rq_last_launch() == ""
     with pytest.raises(rq.RQError, match="RQ_EINVAL"):
         rq.rq_beta_lloyd_max(2, 4)
+
+
+def test_outlier_entry_points_validate_before_launch():
+    import torch
+    k = torch.zeros(64 * 128, dtype=torch.bfloat16)
+    S = torch.zeros(256, 128, dtype=torch.bfloat16)
+    b = torch.zeros(4096, dtype=torch.uint8)
+    n = torch.zeros(64, dtype=torch.int16)
+    ws = torch.zeros(64 * 128 * 2, dtype=torch.uint8)
+    assert rq.qjl_sketch_outlier_workspace_bytes(64, 128) == 64 * 128 * 2
+    for kw, want in ((dict(d=256), "RQ_EUNSUPPORTED"), (dict(d=100), "RQ_EINVAL"), (dict(n_out=0), "RQ_EINVAL"),
+                     (dict(n_out=17), "RQ_EINVAL"), (dict(m_o=48), "RQ_EINVAL"), (dict(m_o=512), "RQ_EINVAL"),
+                     (dict(n_vec=48), "RQ_EINVAL")):
+        a = dict(d=128, m=256, m_o=128, n_out=8, n_vec=64)
+        a.update(kw)
+        with pytest.raises(rq.RQError, match=want):
+            rq.qjl_sketch_outlier(k, a["d"], a["m"], S, a["m_o"], a["n_out"], b, n, b, b, n, ws, stream=0,
+                                  n_vec=a["n_vec"])
+    with pytest.raises(rq.RQError, match="RQ_ESIZE"):
+        rq.qjl_sketch_outlier(k, 128, 256, S, 128, 8, b, n, b, b, n, ws[:100], stream=0)
+    with pytest.raises(rq.RQError, match="RQ_EINVAL"):      # T not a multiple of the group
+        rq.qjl_score_outlier(k, 1, 4, 128, 256, S, b, n, 48, 128, 8, b, b, n, torch.zeros(1), ws, stream=0)
+    assert L.rq_last_launch() == ""
