@@ -59,7 +59,7 @@ def parse(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--profile", default=None,
                    help="run one case's kernels once (profiling driver): c3_layer, weight4096_fused, kv_sketch, "
-                        "kv_score, kv_attention, kv_v, kv_v96, kv_dense, tq256, tq512; print nothing else")
+                        "kv_score, kv_attention, kv_outlier, kv_v, kv_v96, kv_dense, tq256, tq512; print nothing else")
     p.add_argument("--rank-selftest", action="store_true", help=argparse.SUPPRESS)
     return p.parse_args(argv)
 
@@ -425,7 +425,9 @@ def secondary_lines(dev, reps=10, only=None):
     flush = l2_flusher(dev)
     out = []
     # the attention line runs on the key line's sketch, so it comes with it
-    want = (lambda k: True) if only is None else (lambda k: k == only or (only == "kv_k" and k == "kv_attn"))
+    want = (lambda k: True) if only is None else (lambda k: k == only or (only == "kv_k" and k in ("kv_attn",
+                                                                                                   "kv_outlier"))
+                                                  or (only == "kv_outlier" and k == "kv_k"))
 
     if want("c1"):
         # 256 x 512 fp16, d = 128, 4-bit int8 codes, no signs: L2-resident latency
@@ -558,6 +560,30 @@ def secondary_lines(dev, reps=10, only=None):
                     "sketch_roofline": roofline_hbm(kbytes, tk, flops=2 * m * d * G * T),
                     "score_roofline": roofline_hbm(sbytes, ts, note="signs + norms read, fp32 scores written; "
                                                                     "query prologue included")})
+        if want("kv_outlier"):
+            # the same keys with the per-group outlier sketch: 8 outliers per 32 tokens, m_o = 256
+            mo, nout = 256, 8
+            oidx = torch.empty(G * T // 32 * nout, dtype=torch.uint8, device=dev)
+            osg = torch.empty(G * T * mo // 8, dtype=torch.uint8, device=dev)
+            onr = torch.empty(G * T, dtype=torch.int16, device=dev)
+            kin = torch.empty(rq.qjl_sketch_outlier_workspace_bytes(G * T, d), dtype=torch.uint8, device=dev)
+            osk = lambda: rq.qjl_sketch_outlier(k, d, m, S, mo, nout, signs, kn, oidx, osg, onr, kin)
+            osc = lambda: rq.qjl_score_outlier(q, G, nq, d, m, S, signs, kn, T, mo, nout, oidx, osg, onr, scores, ws)
+            osk(); osc()
+            tok_, tos = median_ms(osk, reps, batch=4), median_ms(osc, reps, flush)
+            okbytes = k.numel() * 2 + signs.numel() + osg.numel() + 4 * G * T + oidx.numel()
+            osbytes = sbytes + osg.numel() + 2 * G * T + oidx.numel() + 4 * G * nq * T
+            out.append({"workload": "KV cache K 4x8x32768x128 bf16 (4 channels/head x10): QJL sketch m=256 with the "
+                                    "per-group outlier sketch (8 of 128 coordinates per 32 tokens, m_o=256); score of "
+                                    "32 queries per (batch, head) with the outlier term",
+                        "sketch_ms": round(tok_, 4), "score_ms": round(tos, 4),
+                        "score_tokens_per_s": round(G * T / (tos * 1e-3), 1),
+                        "sketch_roofline": roofline_hbm(okbytes, tok_, note="keys read once; the masked copy's "
+                                                                             "write and re-read are not counted"),
+                        "score_roofline": roofline_hbm(osbytes, tos, note="main and outlier records read, fp32 "
+                                                                          "scores written and re-read")})
+            del oidx, osg, onr, kin
+            sk()                                             # the plain sketch again for the attention line
         del scores, ws
         if want("kv_attn"):
             # attention decode over the sketched keys and the 4-bit values of the V line's recipe
@@ -804,7 +830,7 @@ def profile_case(case):
         rq.rq_dequantize(codes, norms, LAYER_N, D, BITS, rq.RQ_CODES_PACKED, 1, 1000, cent, out)
     else:
         key = {"weight4096_fused": "weight4096", "kv_sketch": "kv_k", "kv_score": "kv_k", "kv_attention": "kv_k",
-               "kv_v": "kv_v", "kv_v96": "kv_v96", "kv_dense": "kv_dense", "tq256": "tq256", "tq512": "tq512"}[case]
+               "kv_v": "kv_v", "kv_v96": "kv_v96", "kv_dense": "kv_dense", "kv_outlier": "kv_outlier", "tq256": "tq256", "tq512": "tq512"}[case]
         secondary_lines(dev, reps=1, only=key)
     torch.cuda.synchronize()
     assert rq.rq_device_error(True) == 0

@@ -17,9 +17,9 @@
 //   its k outlier values, forms ||k_out|| (fp32 squares in stored order) and
 //   the m_o sign bits of sum_r S[i][O_r] v_r (fp32, stored order), and the warp
 //   writes the masked group back contiguously.
-// outlier_score_kernel: one CTA per (head, group): u[q][i] = sum_r S[i][O_r]
-//   q[O_r] for every query, then lane = token adds
-//   sqrt(pi/2)/m_o * n_out16 * sum_i u[q][i] (+1 / -1 by the sign bit) to the
+// outlier_score_kernel: one CTA per (head, group): per token the k weights
+//   w[t][r] = sum_i S[i][O_r] (+1 / -1 by sign bit i), then for every query
+//   lane = token adds sqrt(pi/2)/m_o * n_out16 * sum_r q[O_r] w[t][r] to the
 //   scores the pure-QJL score wrote.
 #include <cmath>
 #include <cstdint>
@@ -129,11 +129,13 @@ outlier_score_kernel(const uint16_t *__restrict__ q, int nq, int64_t T, int m_o,
                      const uint8_t *__restrict__ out_signs, const uint16_t *__restrict__ out_norms,
                      float *__restrict__ scores)
 {
+    // <S_o q_O, s_t> = sum_r q[O_r] w[t][r] with w[t][r] = sum_i S[i][O_r] s_t,i:
+    // the k weights of a token are formed once (m_o signed adds each), and each
+    // (token, query) score then takes k multiply-adds.
     constexpr int d = 128;
-    extern __shared__ float ol_smem[];
-    float *u = ol_smem;                                  // [nq][m_o]
-    __shared__ float so[kOlMaxMo * kOlMaxOut];
-    __shared__ float qo[32 * kOlMaxOut];
+    __shared__ float sct[kOlMaxOut][kOlMaxMo];          // S[i][O_r], transposed
+    __shared__ float w[32][kOlMaxOut + 1];               // per token of the group
+    __shared__ float qo[32][kOlMaxOut + 1];
     __shared__ int sel[kOlMaxOut];
     const int64_t ng = T / 32;
     const int64_t hg = blockIdx.x;                       // (head, group)
@@ -141,35 +143,46 @@ outlier_score_kernel(const uint16_t *__restrict__ q, int nq, int64_t T, int m_o,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < n_out) sel[tid] = idx[hg * n_out + tid];
     __syncthreads();
-    for (int e = tid; e < m_o * n_out; e += blockDim.x) so[e] = bf16_at(S + (int64_t)(e / n_out) * d + sel[e % n_out]);
+    for (int e = tid; e < m_o * n_out; e += blockDim.x) {
+        const int i = e / n_out, r = e - i * n_out;
+        sct[r][i] = bf16_at(S + (int64_t)i * d + sel[r]);
+    }
+    __syncthreads();
+    // weights: warp -> outlier rows r = warp, warp + 4, ...; lane -> token
+    {
+        const int64_t tok = g * T + j * 32 + lane;
+        const uint32_t *sg = reinterpret_cast<const uint32_t *>(out_signs + tok * (m_o / 8));
+        for (int r = warp; r < n_out; r += 4) {
+            const float *col = sct[r];
+            float2 acc = make_float2(0.0f, 0.0f);
+            for (int wd = 0; wd < m_o / 32; ++wd) {
+                const uint32_t bits = __ldg(sg + wd);
+#pragma unroll
+                for (int b = 0; b < 32; b += 2) {
+                    // +S where the bit is set, -S where it is clear
+                    const float x = __uint_as_float(__float_as_uint(col[32 * wd + b]) ^ ((~bits << (31 - b)) & 0x80000000u));
+                    const float y =
+                        __uint_as_float(__float_as_uint(col[32 * wd + b + 1]) ^ ((~bits << (30 - b)) & 0x80000000u));
+                    acc = __fadd2_rn(acc, make_float2(x, y));
+                }
+            }
+            w[lane][r] = __fadd_rn(acc.x, acc.y);
+        }
+    }
     const float c = (float)(1.2533141373155002512 / (double)m_o);   // sqrt(pi/2) / m_o
+    const int64_t tok = g * T + j * 32 + lane;
+    const float no = h16_to_f32(out_norms[tok]) * c;
     for (int q0 = 0; q0 < nq; q0 += 32) {
         const int nqc = nq - q0 < 32 ? nq - q0 : 32;
         __syncthreads();
         for (int e = tid; e < nqc * n_out; e += blockDim.x) {
             const int qq = e / n_out, r = e - qq * n_out;
-            qo[e] = bf16_at(q + (g * nq + q0 + qq) * d + sel[r]);
+            qo[qq][r] = bf16_at(q + (g * nq + q0 + qq) * d + sel[r]);
         }
         __syncthreads();
-        for (int e = tid; e < nqc * m_o; e += blockDim.x) {
-            const int qq = e / m_o, i = e - qq * m_o;
-            float s = 0.0f;
-            for (int r = 0; r < n_out; ++r) s = __fadd_rn(s, __fmul_rn(so[i * n_out + r], qo[qq * n_out + r]));
-            u[e] = s;
-        }
-        __syncthreads();
-        // lane = token of the group, warps stride over the queries
-        const int64_t tok = g * T + j * 32 + lane;
-        const float no = h16_to_f32(out_norms[tok]) * c;
-        const uint8_t *sg = out_signs + tok * (m_o / 8);
-        for (int qq = warp; qq < nqc; qq += blockDim.x / 32) {
-            const float *uq = u + qq * m_o;
+        for (int qq = warp; qq < nqc; qq += 4) {
             float dot = 0.0f;
-            for (int i = 0; i < m_o; i += 8) {
-                const uint32_t byte = sg[i / 8];
-#pragma unroll
-                for (int b = 0; b < 8; ++b) dot = __fadd_rn(dot, ((byte >> b) & 1u) ? uq[i + b] : -uq[i + b]);
-            }
+            for (int r = 0; r < n_out; ++r) dot = __fadd_rn(dot, __fmul_rn(qo[qq][r], w[lane][r]));
             float *dst = scores + (g * nq + q0 + qq) * T + j * 32 + lane;
             *dst = __fadd_rn(*dst, __fmul_rn(no, dot));
         }
@@ -178,7 +191,6 @@ outlier_score_kernel(const uint16_t *__restrict__ q, int nq, int64_t T, int m_o,
 
 }  // namespace
 
-size_t outlier_score_smem(int nq, int m_o) { return (size_t)(nq < 32 ? nq : 32) * m_o * 4; }
 
 cudaError_t launch_outlier_prep(const uint16_t *keys, int64_t nvec, int n_out, int m_o, const uint16_t *S,
                                 uint16_t *kin, uint8_t *idx, uint8_t *out_signs, uint16_t *out_norms, int num_sms,
@@ -201,11 +213,8 @@ cudaError_t launch_outlier_score(const uint16_t *q, int64_t G, int nq, int64_t T
                                  const uint16_t *S, const uint8_t *idx, const uint8_t *out_signs,
                                  const uint16_t *out_norms, float *scores, cudaStream_t st)
 {
-    const size_t smem = outlier_score_smem(nq, m_o);
-    cudaError_t e = cudaFuncSetAttribute(outlier_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const int64_t blocks = G * (T / 32);
-    outlier_score_kernel<<<(unsigned)blocks, 128, smem, st>>>(q, nq, T, m_o, n_out, S, idx, out_signs, out_norms,
+    outlier_score_kernel<<<(unsigned)blocks, 128, 0, st>>>(q, nq, T, m_o, n_out, S, idx, out_signs, out_norms,
                                                              scores);
     note_launch("outlier_score_kernel");
     return cudaGetLastError();
