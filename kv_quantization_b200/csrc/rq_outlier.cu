@@ -85,10 +85,18 @@ outlier_prep_kernel(const uint16_t *__restrict__ keys, int64_t ngroups, int n_ou
             }
         }
         __syncwarp();
-        // S columns of the outlier set
-        for (int e = lane; e < m_o * n_out; e += 32) {
-            const int i = e / n_out, r = e - i * n_out;
-            sow[e] = bf16_at(S + (int64_t)i * d + sel[warp][r]);
+        // S columns of the outlier set: eight independent gathers in flight per lane
+        for (int e0 = 0; e0 < m_o * n_out; e0 += 256) {
+            float g8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + lane + 32 * u;
+                const int i = e / n_out, r = e - i * n_out;
+                g8[u] = e < m_o * n_out ? bf16_at(S + (int64_t)i * d + sel[warp][r]) : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (e0 + lane + 32 * u < m_o * n_out) sow[e0 + lane + 32 * u] = g8[u];
         }
         // lane = token: outlier values, norm, sketch
         float v[kOlMaxOut];
