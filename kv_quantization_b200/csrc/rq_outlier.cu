@@ -37,8 +37,9 @@ constexpr int kOlMaxMo = 256;
 
 __device__ __forceinline__ float bf16_at(const uint16_t *p) { return __uint_as_float((uint32_t)*p << 16); }
 
+template <int NOUT>
 __global__ void __launch_bounds__(kOlWarps * 32)
-outlier_prep_kernel(const uint16_t *__restrict__ keys, int64_t ngroups, int n_out, int m_o,
+outlier_prep_kernel(const uint16_t *__restrict__ keys, int64_t ngroups, int m_o,
                     const uint16_t *__restrict__ S, uint16_t *__restrict__ kin, uint8_t *__restrict__ idx_out,
                     uint8_t *__restrict__ out_signs, uint16_t *__restrict__ out_norms)
 {
@@ -46,8 +47,8 @@ outlier_prep_kernel(const uint16_t *__restrict__ keys, int64_t ngroups, int n_ou
     extern __shared__ __align__(16) uint8_t ol_prep_smem[];
     __shared__ int sel[kOlWarps][kOlMaxOut];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // per warp: the group's keys (8 KB), then S[i][O_r] for i < m_o (m_o * n_out floats)
-    uint8_t *wb = ol_prep_smem + (size_t)warp * (32 * d * 2 + (size_t)m_o * n_out * 4);
+    // per warp: the group's keys (8 KB), then S[i][O_r] as [r][i] (NOUT * m_o floats)
+    uint8_t *wb = ol_prep_smem + (size_t)warp * (32 * d * 2 + (size_t)m_o * NOUT * 4);
     uint16_t *tl = reinterpret_cast<uint16_t *>(wb);
     float *sow = reinterpret_cast<float *>(wb + 32 * d * 2);
     for (int64_t g = (int64_t)blockIdx.x * kOlWarps + warp; g < ngroups; g += (int64_t)gridDim.x * kOlWarps) {
@@ -66,7 +67,7 @@ outlier_prep_kernel(const uint16_t *__restrict__ keys, int64_t ngroups, int n_ou
             }
         // top n_out: largest sum first, ties to the lower column
         uint32_t taken = 0u;
-        for (int r = 0; r < n_out; ++r) {
+        for (int r = 0; r < NOUT; ++r) {
             float bv = -1.0f;
             int bi = 1 << 30;
 #pragma unroll
@@ -81,49 +82,45 @@ outlier_prep_kernel(const uint16_t *__restrict__ keys, int64_t ngroups, int n_ou
             if ((bi >> 2) == lane) taken |= 1u << (bi & 3);
             if (lane == 0) {
                 sel[warp][r] = bi;
-                idx_out[g * n_out + r] = (uint8_t)bi;
+                idx_out[g * NOUT + r] = (uint8_t)bi;
             }
         }
         __syncwarp();
-        // S columns of the outlier set: eight independent gathers in flight per lane
-        for (int e0 = 0; e0 < m_o * n_out; e0 += 256) {
-            float g8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + lane + 32 * u;
-                const int i = e / n_out, r = e - i * n_out;
-                g8[u] = e < m_o * n_out ? bf16_at(S + (int64_t)i * d + sel[warp][r]) : 0.0f;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (e0 + lane + 32 * u < m_o * n_out) sow[e0 + lane + 32 * u] = g8[u];
+        // S columns of the outlier set, transposed: sow[r][i] = S[i][O_r]
+        for (int e = lane; e < m_o * NOUT; e += 32) {
+            const int r = e / m_o, i = e - r * m_o;
+            sow[e] = bf16_at(S + (int64_t)i * d + sel[warp][r]);
         }
         // lane = token: outlier values, norm, sketch
-        float v[kOlMaxOut];
+        float v[NOUT];
         float acc = 0.0f;
 #pragma unroll
-        for (int r = 0; r < kOlMaxOut; ++r) {
-            v[r] = r < n_out ? bf16_at(tl + lane * d + sel[warp][r]) : 0.0f;
-            if (r < n_out) acc = __fadd_rn(acc, __fmul_rn(v[r], v[r]));
+        for (int r = 0; r < NOUT; ++r) {
+            v[r] = bf16_at(tl + lane * d + sel[warp][r]);
+            acc = __fadd_rn(acc, __fmul_rn(v[r], v[r]));
         }
         const int64_t tok = g * 32 + lane;
         out_norms[tok] = norm_to_h16(__fsqrt_rn(acc));
         __syncwarp();
         for (int w = 0; w < m_o / 32; ++w) {
             uint32_t bits = 0u;
-            for (int b = 0; b < 32; ++b) {
-                const float *row = sow + (32 * w + b) * n_out;
-                float p = 0.0f;
+#pragma unroll 4
+            for (int b = 0; b < 32; b += 2) {              // outputs i, i + 1 as a pair
+                const int i = 32 * w + b;
+                float2 p = make_float2(0.0f, 0.0f);
 #pragma unroll
-                for (int r = 0; r < kOlMaxOut; ++r)
-                    if (r < n_out) p = __fadd_rn(p, __fmul_rn(row[r], v[r]));
-                bits |= (p >= 0.0f ? 1u : 0u) << b;
+                for (int r = 0; r < NOUT; ++r) {
+                    const float2 sv = *reinterpret_cast<const float2 *>(sow + r * m_o + i);
+                    p = __fadd2_rn(p, __fmul2_rn(sv, make_float2(v[r], v[r])));
+                }
+                bits |= (p.x >= 0.0f ? 1u : 0u) << b;
+                bits |= (p.y >= 0.0f ? 1u : 0u) << (b + 1);
             }
             reinterpret_cast<uint32_t *>(out_signs + tok * (m_o / 8))[w] = bits;
         }
         // masked group back, contiguous
         __syncwarp();
-        for (int r = 0; r < n_out; ++r) tl[lane * d + sel[warp][r]] = 0;
+        for (int r = 0; r < NOUT; ++r) tl[lane * d + sel[warp][r]] = 0;
         __syncwarp();
         uint4 *dst = reinterpret_cast<uint4 *>(kin + g * 32 * d);
 #pragma unroll
@@ -200,21 +197,40 @@ outlier_score_kernel(const uint16_t *__restrict__ q, int nq, int64_t T, int m_o,
 }  // namespace
 
 
+template <int NOUT>
+static cudaError_t run_outlier_prep(const uint16_t *keys, int64_t ngroups, int m_o, const uint16_t *S, uint16_t *kin,
+                                    uint8_t *idx, uint8_t *out_signs, uint16_t *out_norms, int num_sms, cudaStream_t st)
+{
+    int64_t grid = (ngroups + kOlWarps - 1) / kOlWarps;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (grid > cap) grid = cap;
+    const size_t smem = (size_t)kOlWarps * (32 * 128 * 2 + (size_t)m_o * NOUT * 4);
+    cudaError_t e = cudaFuncSetAttribute(outlier_prep_kernel<NOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    outlier_prep_kernel<NOUT><<<(unsigned)(grid > 0 ? grid : 1), kOlWarps * 32, smem, st>>>(keys, ngroups, m_o, S, kin,
+                                                                                           idx, out_signs, out_norms);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_outlier_prep(const uint16_t *keys, int64_t nvec, int n_out, int m_o, const uint16_t *S,
                                 uint16_t *kin, uint8_t *idx, uint8_t *out_signs, uint16_t *out_norms, int num_sms,
                                 cudaStream_t st)
 {
-    const int64_t ngroups = nvec / 32;
-    int64_t grid = (ngroups + kOlWarps - 1) / kOlWarps;
-    const int64_t cap = (int64_t)num_sms * 8;
-    if (grid > cap) grid = cap;
-    const size_t smem = (size_t)kOlWarps * (32 * 128 * 2 + (size_t)m_o * n_out * 4);
-    cudaError_t e = cudaFuncSetAttribute(outlier_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    outlier_prep_kernel<<<(unsigned)(grid > 0 ? grid : 1), kOlWarps * 32, smem, st>>>(keys, ngroups, n_out, m_o, S,
-                                                                                     kin, idx, out_signs, out_norms);
+    const int64_t ng = nvec / 32;
+    cudaError_t e;
+    switch (n_out) {
+#define RQ_OUTLIER_CASE(K) \
+    case K: e = run_outlier_prep<K>(keys, ng, m_o, S, kin, idx, out_signs, out_norms, num_sms, st); break;
+        RQ_OUTLIER_CASE(1) RQ_OUTLIER_CASE(2) RQ_OUTLIER_CASE(3) RQ_OUTLIER_CASE(4) RQ_OUTLIER_CASE(5)
+        RQ_OUTLIER_CASE(6) RQ_OUTLIER_CASE(7) RQ_OUTLIER_CASE(8) RQ_OUTLIER_CASE(9) RQ_OUTLIER_CASE(10)
+        RQ_OUTLIER_CASE(11) RQ_OUTLIER_CASE(12) RQ_OUTLIER_CASE(13) RQ_OUTLIER_CASE(14) RQ_OUTLIER_CASE(15)
+        RQ_OUTLIER_CASE(16)
+#undef RQ_OUTLIER_CASE
+    default: return cudaErrorNotSupported;
+    }
     note_launch("outlier_prep_kernel");
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_outlier_score(const uint16_t *q, int64_t G, int nq, int64_t T, int m_o, int n_out,
